@@ -1,0 +1,300 @@
+// Host side of the LazyFlash C ABI (include/lazyflash.h): argument checks,
+// workspace sizing, TMA tensor-map encoding and kernel launches.  Nothing
+// here computes attention; every step of the path runs in the kernels of
+// lf_fwd.cuh, lf_select.cuh and lf_bwd.cuh.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "lazyflash.h"
+#include "lf_bwd.cuh"
+#include "lf_device.cuh"
+#include "lf_fwd.cuh"
+#include "lf_select.cuh"
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q{};
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+lf_status check_desc(const lf_attn_desc* d) {
+    if (!d) return LF_ERR_INVALID_ARG;
+    if (d->nseq < 1 || !d->cu_seqlens || d->total_tokens < 0 || d->max_seqlen < 0)
+        return LF_ERR_INVALID_ARG;
+    if (d->hq < 1 || d->hkv < 1 || d->hq % d->hkv != 0) return LF_ERR_INVALID_ARG;
+    if (d->hq > 65535 || d->hkv > 65535) return LF_ERR_UNSUPPORTED;
+    if (!(d->softmax_scale > 0.f) || !std::isfinite(d->softmax_scale)) return LF_ERR_INVALID_ARG;
+    if (d->causal != 0 && d->causal != 1) return LF_ERR_INVALID_ARG;
+    if (d->d != 64 && d->d != 128) return LF_ERR_UNSUPPORTED;
+    if (d->block_q != 64 && d->block_q != 128) return LF_ERR_UNSUPPORTED;
+    if (d->nseq > 65535) return LF_ERR_UNSUPPORTED;
+    // element offsets are computed in 64 bits; row indices in 32 bits
+    if ((int64_t)d->total_tokens * d->hq > (int64_t)1 << 31) return LF_ERR_UNSUPPORTED;
+    return LF_OK;
+}
+
+inline int nbmax_of(const lf_attn_desc* d) { return (d->max_seqlen + d->block_q - 1) / d->block_q; }
+inline int ntiles_of(const lf_attn_desc* d) { return (d->max_seqlen + 127) / 128; }
+
+size_t bwd_ws_bytes(const lf_attn_desc* d, bool need_D) {
+    size_t b = (size_t)d->total_tokens * d->hq * d->d * sizeof(float);   // fp32 dQ accumulator
+    b = (b + 255) & ~size_t(255);
+    if (need_D) b += ((size_t)d->total_tokens * d->hq * sizeof(float) + 255) & ~size_t(255);
+    return b;
+}
+
+// [T][H][d] bf16 -> 3-D map (d, H, T), 64 x 1 x 128 boxes, 128-byte swizzle.
+bool make_thd_map(CUtensorMap* m, const void* base, int T, int H, int D) {
+    EncodeTiledFn enc = encode_tiled();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
+    const cuuint32_t box[3] = {64, 1, 128};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
+               estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline lf_status launch_status() {
+    return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
+}
+
+template <int D>
+lf_status launch_fwd(const lf_attn_desc* d, const void* q, const void* k, const void* v, void* o,
+                     float* lse, cudaStream_t st) {
+    CUtensorMap mq, mk, mv;
+    if (!make_thd_map(&mq, q, d->total_tokens, d->hq, D) ||
+        !make_thd_map(&mk, k, d->total_tokens, d->hkv, D) ||
+        !make_thd_map(&mv, v, d->total_tokens, d->hkv, D))
+        return LF_ERR_CUDA;
+    lf::FwdParams p{};
+    p.cu_seqlens = d->cu_seqlens;
+    p.T = d->total_tokens;
+    p.hq = d->hq;
+    p.hkv = d->hkv;
+    p.causal = d->causal;
+    p.max_seqlen = d->max_seqlen;
+    p.scale_log2 = d->softmax_scale * 1.4426950408889634f;
+    p.o = static_cast<__nv_bfloat16*>(o);
+    p.lse = lse;
+    const uint32_t smem = lf::FwdSmem<D>::kAlloc;
+    if (cudaFuncSetAttribute(lf::attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+        return LF_ERR_CUDA;
+    dim3 grid(d->hq, ntiles_of(d), d->nseq);
+    lf::attn_fwd_kernel<D><<<grid, lf::kFwdThreads, smem, st>>>(mq, mk, mv, p);
+    return launch_status();
+}
+
+template <int D>
+lf_status launch_norms(const lf_attn_desc* d, const void* dout, const void* o, float* norms,
+                       float* Dv, int write_norms, cudaStream_t st) {
+    dim3 grid(nbmax_of(d), d->hq, d->nseq);
+    lf::norms_rowdot_kernel<D><<<grid, 128, 0, st>>>(
+        d->cu_seqlens, d->total_tokens, d->max_seqlen, d->hq, d->block_q, nbmax_of(d),
+        static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(o), norms, Dv,
+        write_norms);
+    return launch_status();
+}
+
+template <int D>
+lf_status launch_bwd(const lf_attn_desc* d, const void* q, const void* k, const void* v,
+                     const float* lse, const void* dout, const float* Dv, const float* w,
+                     const int32_t* kidx, const int32_t* kcnt, void* dq, void* dk, void* dv,
+                     float* dq_acc, cudaStream_t st) {
+    CUtensorMap mq, mk, mv, mdo;
+    if (!make_thd_map(&mq, q, d->total_tokens, d->hq, D) ||
+        !make_thd_map(&mk, k, d->total_tokens, d->hkv, D) ||
+        !make_thd_map(&mv, v, d->total_tokens, d->hkv, D) ||
+        !make_thd_map(&mdo, dout, d->total_tokens, d->hq, D))
+        return LF_ERR_CUDA;
+    const size_t nacc = (size_t)d->total_tokens * d->hq * D;
+    if (cudaMemsetAsync(dq_acc, 0, nacc * sizeof(float), st) != cudaSuccess) return LF_ERR_CUDA;
+    lf::BwdParams p{};
+    p.cu_seqlens = d->cu_seqlens;
+    p.T = d->total_tokens;
+    p.hq = d->hq;
+    p.hkv = d->hkv;
+    p.causal = d->causal;
+    p.block_q = d->block_q;
+    p.nbmax = nbmax_of(d);
+    p.max_seqlen = d->max_seqlen;
+    p.scale = d->softmax_scale;
+    p.scale_log2 = d->softmax_scale * 1.4426950408889634f;
+    p.lse = lse;
+    p.Dvec = Dv;
+    p.block_weight = w;
+    p.kept_idx = kidx;
+    p.kept_cnt = kcnt;
+    p.dq_acc = dq_acc;
+    p.dk = static_cast<__nv_bfloat16*>(dk);
+    p.dv = static_cast<__nv_bfloat16*>(dv);
+    const uint32_t smem = lf::BwdSmem<D>::kAlloc;
+    if (cudaFuncSetAttribute(lf::attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             smem) != cudaSuccess)
+        return LF_ERR_CUDA;
+    dim3 grid(d->hkv, ntiles_of(d), d->nseq);
+    lf::attn_bwd_kernel<D><<<grid, lf::kBwdThreads, smem, st>>>(mq, mk, mv, mdo, p);
+    if (launch_status() != LF_OK) return LF_ERR_CUDA;
+    const size_t n8 = nacc / 8;
+    const int blocks = (int)std::min<size_t>((n8 + 255) / 256, 148 * 16);
+    lf::dq_convert_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(dq_acc),
+                                                  static_cast<uint4*>(dq), n8, d->softmax_scale);
+    return launch_status();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* lf_status_string(lf_status s) {
+    switch (s) {
+        case LF_OK: return "LF_OK";
+        case LF_ERR_INVALID_ARG: return "LF_ERR_INVALID_ARG: invalid argument";
+        case LF_ERR_UNSUPPORTED: return "LF_ERR_UNSUPPORTED: shape not supported by this build";
+        case LF_ERR_WORKSPACE: return "LF_ERR_WORKSPACE: workspace too small";
+        case LF_ERR_CUDA: return "LF_ERR_CUDA: CUDA call failed";
+        case LF_ERR_TIMEOUT: return "LF_ERR_TIMEOUT: a device-side bounded wait expired";
+    }
+    return "unknown lf_status";
+}
+
+lf_status lf_workspace_size(const lf_attn_desc* desc, int which, size_t* bytes) {
+    lf_status st = check_desc(desc);
+    if (st != LF_OK) return st;
+    if (!bytes) return LF_ERR_INVALID_ARG;
+    switch (which) {
+        case LF_WS_FWD: *bytes = 0; return LF_OK;
+        case LF_WS_SELECT: *bytes = 0; return LF_OK;
+        case LF_WS_BWD: *bytes = bwd_ws_bytes(desc, true); return LF_OK;
+    }
+    return LF_ERR_INVALID_ARG;
+}
+
+lf_status lf_attn_fwd(const lf_attn_desc* desc, const void* q, const void* k, const void* v,
+                      void* o, float* lse, void* ws, size_t ws_bytes, lf_stream_t stream) {
+    (void)ws;
+    (void)ws_bytes;
+    lf_status st = check_desc(desc);
+    if (st != LF_OK) return st;
+    if (!q || !k || !v || !o || !lse) return LF_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+        return LF_ERR_INVALID_ARG;
+    if (desc->total_tokens == 0 || desc->max_seqlen == 0) return LF_OK;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    return desc->d == 128 ? launch_fwd<128>(desc, q, k, v, o, lse, s)
+                          : launch_fwd<64>(desc, q, k, v, o, lse, s);
+}
+
+lf_status lf_block_select(const lf_attn_desc* desc, const void* dout, const void* o, double delta,
+                          uint64_t seed, uint64_t step, uint32_t flags, float* block_norm,
+                          float* D, double* tau, float* block_weight, uint8_t* keep,
+                          int32_t* kept_idx, int32_t* kept_cnt, void* ws, size_t ws_bytes,
+                          lf_stream_t stream) {
+    (void)ws;
+    (void)ws_bytes;
+    lf_status st = check_desc(desc);
+    if (st != LF_OK) return st;
+    if (!(delta >= 0.0 && delta < 1.0)) return LF_ERR_INVALID_ARG;
+    if (flags & ~LF_SELECT_NORMS_GIVEN) return LF_ERR_INVALID_ARG;
+    if (!dout || !o || !block_norm || !D || !tau || !block_weight || !keep || !kept_idx ||
+        !kept_cnt)
+        return LF_ERR_INVALID_ARG;
+    if (!aligned16(dout) || !aligned16(o) || !aligned16(block_norm) || !aligned16(D) ||
+        !aligned16(tau) || !aligned16(block_weight) || !aligned16(keep) || !aligned16(kept_idx) ||
+        !aligned16(kept_cnt))
+        return LF_ERR_INVALID_ARG;
+    if (desc->max_seqlen == 0) return LF_OK;
+    const int nbmax = nbmax_of(desc);
+    if ((size_t)nbmax * sizeof(double) > 200 * 1024) return LF_ERR_UNSUPPORTED;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int write_norms = (flags & LF_SELECT_NORMS_GIVEN) ? 0 : 1;
+    st = desc->d == 128 ? launch_norms<128>(desc, dout, o, block_norm, D, write_norms, s)
+                        : launch_norms<64>(desc, dout, o, block_norm, D, write_norms, s);
+    if (st != LF_OK) return st;
+    const size_t smem = (size_t)nbmax * sizeof(double);
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(lf::select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return LF_ERR_CUDA;
+    dim3 grid(desc->hq, desc->nseq);
+    lf::select_kernel<<<grid, 32, smem, s>>>(desc->cu_seqlens, desc->total_tokens,
+                                             desc->max_seqlen, desc->hq, desc->block_q, nbmax,
+                                             block_norm, delta, seed, step, tau, block_weight,
+                                             keep, kept_idx, kept_cnt);
+    return launch_status();
+}
+
+lf_status lf_attn_bwd(const lf_attn_desc* desc, const void* q, const void* k, const void* v,
+                      const void* o, const float* lse, const void* dout, const float* D,
+                      const float* block_weight, const int32_t* kept_idx,
+                      const int32_t* kept_cnt, void* dq, void* dk, void* dv, void* ws,
+                      size_t ws_bytes, lf_stream_t stream) {
+    lf_status st = check_desc(desc);
+    if (st != LF_OK) return st;
+    if (!q || !k || !v || !lse || !dout || !block_weight || !kept_idx || !kept_cnt || !dq ||
+        !dk || !dv)
+        return LF_ERR_INVALID_ARG;
+    if (!D && !o) return LF_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, lse, dout, block_weight, kept_idx, kept_cnt, dq, dk, dv, ws};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return LF_ERR_INVALID_ARG;
+    if ((o && !aligned16(o)) || (D && !aligned16(D))) return LF_ERR_INVALID_ARG;
+    if (desc->total_tokens == 0 || desc->max_seqlen == 0) return LF_OK;
+    if (!ws || ws_bytes < bwd_ws_bytes(desc, D == nullptr)) return LF_ERR_WORKSPACE;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    float* dq_acc = static_cast<float*>(ws);
+    const float* Dv = D;
+    if (!Dv) {
+        const size_t acc = ((size_t)desc->total_tokens * desc->hq * desc->d * sizeof(float) + 255) &
+                           ~size_t(255);
+        float* Dw = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + acc);
+        st = desc->d == 128 ? launch_norms<128>(desc, dout, o, nullptr, Dw, 0, s)
+                            : launch_norms<64>(desc, dout, o, nullptr, Dw, 0, s);
+        if (st != LF_OK) return st;
+        Dv = Dw;
+    }
+    return desc->d == 128 ? launch_bwd<128>(desc, q, k, v, lse, dout, Dv, block_weight, kept_idx,
+                                            kept_cnt, dq, dk, dv, dq_acc, s)
+                          : launch_bwd<64>(desc, q, k, v, lse, dout, Dv, block_weight, kept_idx,
+                                           kept_cnt, dq, dk, dv, dq_acc, s);
+}
+
+lf_status lf_check_device_error(lf_stream_t stream) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return LF_ERR_CUDA;
+    int flag = 0;
+    if (cudaMemcpyFromSymbol(&flag, lf::g_device_error, sizeof(int)) != cudaSuccess)
+        return LF_ERR_CUDA;
+    if (flag == 0) return LF_OK;
+    const int zero = 0;
+    if (cudaMemcpyToSymbol(lf::g_device_error, &zero, sizeof(int)) != cudaSuccess)
+        return LF_ERR_CUDA;
+    return (flag & 0xff) == lf::kErrTimeout ? LF_ERR_TIMEOUT : LF_ERR_INVALID_ARG;
+}
+
+}  // extern "C"

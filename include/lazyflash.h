@@ -1,0 +1,147 @@
+/*
+ * lazyflash.h -- C ABI of the LazyFlash attention hot path on B200 (sm_100a).
+ *
+ * LazyFlash ("LazyFlash allège la rétropropagation de l'attention, 5,72 fois",
+ * gyom.fr, 26 Oct 2026) keeps the attention forward exactly dense and makes
+ * only the backward block-sparse: query blocks are ranked by the norm of their
+ * output gradient, a budget delta bounds the share of gradient mass that may be
+ * discarded, each block is kept with probability proportional to its gradient,
+ * kept blocks are reweighted so the gradient stays unbiased, and dropped tiles
+ * are never loaded or computed.
+ *
+ * Three calls make up one training step of one attention layer:
+ *   lf_attn_fwd      dense forward: O and the per-row log-sum-exp;
+ *   lf_block_select  block norms ||dO_b||, D = rowsum(dO * O), the budgeted
+ *                    threshold tau, the random keep mask, the 1/p weights and
+ *                    the compacted kept-block lists;
+ *   lf_attn_bwd      the backward over kept query blocks only.
+ *
+ * Conventions shared by every call
+ *   Layout ("THD"): every token tensor is [T][H][d] row-major and contiguous,
+ *     bf16 (q, o, dout, dq: H = hq; k, v, dk, dv: H = hkv).  Segments (packed
+ *     variable-length sequences) are delimited by cu_seqlens: int32, nseq + 1
+ *     entries, cu_seqlens[0] = 0, non-decreasing, cu_seqlens[nseq] =
+ *     total_tokens.  Attention never crosses a segment; with causal != 0 key u
+ *     is visible to query t iff u <= t within the segment.
+ *   Query head h reads KV head h / (hq / hkv) (consecutive groups, GQA).
+ *   lse and D are fp32 [hq][T].  Per-block arrays are [nseq][hq][nbmax] with
+ *     nbmax = ceil(max_seqlen / block_q); block i of segment s covers rows
+ *     cu_seqlens[s] + i*block_q ... (the last block of a segment may be short);
+ *     entries past a segment's block count are written as 0 (kept_idx: -1).
+ *   Pointers: all tensor pointers are DEVICE pointers owned by the caller, and
+ *     must be 16-byte aligned.  The library allocates no memory and keeps no
+ *     per-call state; scratch memory is the caller's workspace (ws, ws_bytes),
+ *     sized by lf_workspace_size.
+ *   Ordering: every call only enqueues work on `stream` and returns.
+ *   Errors: argument errors are returned synchronously, before anything is
+ *     launched (LF_ERR_INVALID_ARG, LF_ERR_UNSUPPORTED, LF_ERR_WORKSPACE).
+ *     A failed launch returns LF_ERR_CUDA.  A kernel whose bounded wait expired
+ *     records it in a device flag instead of hanging; lf_check_device_error
+ *     synchronizes the stream and returns LF_ERR_TIMEOUT in that case.
+ *   Thread safety: calls are reentrant; concurrent calls on different streams
+ *     must use different workspaces and outputs.
+ */
+#ifndef LAZYFLASH_H
+#define LAZYFLASH_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* lf_stream_t; /* a cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+    LF_OK = 0,
+    LF_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, inconsistent sizes, delta outside [0,1) */
+    LF_ERR_UNSUPPORTED = 2,  /* a shape this build does not implement (d, block_q) */
+    LF_ERR_WORKSPACE = 3,    /* ws_bytes below lf_workspace_size() */
+    LF_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
+    LF_ERR_TIMEOUT = 5       /* a device-side bounded wait expired (see lf_check_device_error) */
+} lf_status;
+
+typedef struct {
+    int32_t nseq;               /* number of packed segments, >= 1 */
+    const int32_t* cu_seqlens;  /* DEVICE pointer, nseq + 1 int32 offsets */
+    int32_t max_seqlen;         /* >= the longest segment (host value) */
+    int32_t total_tokens;       /* T = cu_seqlens[nseq] (host value), >= 0 */
+    int32_t hq, hkv, d;         /* query heads, KV heads (hq % hkv == 0), head dim (64 or 128) */
+    float softmax_scale;        /* scores are softmax_scale * <q, k>; usually 1/sqrt(d) */
+    int32_t causal;             /* 1: causal within each segment; 0: full within each segment */
+    int32_t block_q;            /* query rows per selection block: 64 or 128 */
+} lf_attn_desc;
+
+enum { LF_WS_FWD = 0, LF_WS_SELECT = 1, LF_WS_BWD = 2 };
+
+/* Flags of lf_block_select. */
+#define LF_SELECT_NORMS_GIVEN 0x1u  /* block_norm is an input; the norm pass only computes D */
+
+/* Bytes of workspace the call `which` (LF_WS_*) needs for `desc`.
+ * Returns LF_ERR_INVALID_ARG / LF_ERR_UNSUPPORTED for a bad descriptor. */
+lf_status lf_workspace_size(const lf_attn_desc* desc, int which, size_t* bytes);
+
+/* Dense attention forward (the LazyFlash forward is FlashAttention's,
+ * unchanged: article standfirst and section "Le passage arrière fait deux fois
+ * le travail du passage avant").
+ *   q [T][hq][d], k, v [T][hkv][d] bf16 in; o [T][hq][d] bf16 out;
+ *   lse [hq][T] fp32 out: natural-log log-sum-exp of softmax_scale * <q_t, k_u>
+ *   over the keys row t sees.
+ *   Rows of o/lse outside every segment are left untouched. */
+lf_status lf_attn_fwd(const lf_attn_desc* desc, const void* q, const void* k, const void* v,
+                      void* o, float* lse, void* ws, size_t ws_bytes, lf_stream_t stream);
+
+/* LazyFlash selection (article section "Un budget sur la masse de gradient, et
+ * un tirage qui garde le gradient non biaisé"), per (segment s, head h):
+ *   block_norm[s][h][i] = ||dO rows of block i||_F (fp32 accumulation; an input
+ *     when flags has LF_SELECT_NORMS_GIVEN);
+ *   D[h][t] = sum_c dO[t][h][c] * O[t][h][c] (fp32, unweighted);
+ *   tau[s][h] (fp64) = the largest threshold whose expected discarded mass
+ *     sum_i (1 - min(1, m_i/tau)) m_i is <= delta * sum_i m_i, found by 64
+ *     bisection steps on [0, max_i m_i / (1 - delta)] with a fixed fp64
+ *     summation order; 0 when delta == 0 or all norms are 0 (keep all);
+ *   p_i = min(1, m_i / tau) (1 when tau == 0); keep_i = 1 iff p_i >= 1 or
+ *     u24 < p_i * 2^24, u24 = word 0 of Philox4x32-10(counter = (i, h, s,
+ *     step mod 2^32), key = (seed lo 32, seed hi 32)) >> 8;
+ *   block_weight[s][h][i] = (float)(1 / p_i) if kept else 0;
+ *   keep (uint8), kept_idx (int32, ascending kept block indices, -1 padded),
+ *   kept_cnt[s][h] (int32).
+ *   delta must lie in [0, 1).  dout and o are [T][hq][d] bf16. */
+lf_status lf_block_select(const lf_attn_desc* desc, const void* dout, const void* o,
+                          double delta, uint64_t seed, uint64_t step, uint32_t flags,
+                          float* block_norm, float* D, double* tau, float* block_weight,
+                          uint8_t* keep, int32_t* kept_idx, int32_t* kept_cnt,
+                          void* ws, size_t ws_bytes, lf_stream_t stream);
+
+/* LazyFlash backward over kept query blocks (article sections "Le passage
+ * arrière ..." and "Un budget sur la masse de gradient ...": dropped tiles are
+ * never loaded or computed; kept blocks' output gradient is scaled by
+ * block_weight).  With dO~ = w_b(t) dO_t and P the softmax of the forward:
+ *   dP = dO~ V^T, dS = P * (dP - w D), dQ = scale dS K, dK = scale dS^T Q
+ *   (summed over the hq/hkv query heads of a KV head), dV = P^T dO~.
+ *   q, k, v, dout bf16 in (layouts as above); lse, D fp32 [hq][T] from
+ *   lf_attn_fwd / lf_block_select (D may be NULL: it is then computed from o
+ *   and dout into the workspace; o may be NULL when D is given);
+ *   block_weight, kept_idx, kept_cnt from lf_block_select;
+ *   dq [T][hq][d], dk, dv [T][hkv][d] bf16 out.  Rows of dropped blocks get
+ *   dq = 0; dk/dv rows no kept block reaches get 0. */
+lf_status lf_attn_bwd(const lf_attn_desc* desc, const void* q, const void* k, const void* v,
+                      const void* o, const float* lse, const void* dout, const float* D,
+                      const float* block_weight, const int32_t* kept_idx,
+                      const int32_t* kept_cnt, void* dq, void* dk, void* dv,
+                      void* ws, size_t ws_bytes, lf_stream_t stream);
+
+/* Waits for `stream`, then reads and clears the device watchdog flag.
+ * LF_ERR_TIMEOUT if a kernel gave up a bounded wait since the last check,
+ * LF_ERR_CUDA if the stream reported an error, else LF_OK. */
+lf_status lf_check_device_error(lf_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+const char* lf_status_string(lf_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LAZYFLASH_H */

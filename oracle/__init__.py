@@ -65,6 +65,11 @@ def lib():
                                      ctypes.POINTER(ctypes.c_uint8), i32p, i32p]
             L.lfo_attn_bwd.argtypes = [c_int, i32p, c_int, c_int, c_int, c_int, c_dbl, c_int,
                                        c_int, c_int, dp, dp, dp, dp, dp, dp, dp, dp]
+            L.lfo_attn_fwd_rows.argtypes = [c_int, i32p, c_int, c_int, c_int, c_int, c_dbl, c_int,
+                                            dp, dp, dp, c_int, i32p, i32p, dp, dp]
+            L.lfo_attn_bwd_rows.argtypes = [c_int, i32p, c_int, c_int, c_int, c_int, c_dbl, c_int,
+                                            c_int, c_int, dp, dp, dp, dp, dp,
+                                            c_int, i32p, i32p, dp, c_int, i32p, i32p, dp, dp]
             _lib = L
     return _lib
 
@@ -207,4 +212,49 @@ def attn_bwd(cu_seqlens, q, k, v, dout, scale: float, block: int, wblk=None,
     _check(lib().lfo_attn_bwd(len(cu) - 1, _p(cu, ctypes.c_int32), T, hq, hkv, d, scale, int(causal),
                               block, nbmax, _p(q, dp), _p(k, dp), _p(v, dp), _p(do, dp), wptr,
                               _p(dq, dp), _p(dk, dp), _p(dv, dp)), "attn_bwd")
+    return dq, dk, dv
+
+
+def attn_fwd_rows(cu_seqlens, q, k, v, scale: float, rows, heads, causal: bool = True):
+    """O [n, d] and LSE [n] of query rows (rows[i], heads[i]) only."""
+    cu = _i32(cu_seqlens)
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    T, hq, d = q.shape
+    hkv = k.shape[1]
+    rows, heads = _i32(rows), _i32(heads)
+    n = len(rows)
+    o = np.zeros((n, d), dtype=np.float64)
+    lse = np.zeros(n, dtype=np.float64)
+    dp, ip = ctypes.c_double, ctypes.c_int32
+    _check(lib().lfo_attn_fwd_rows(len(cu) - 1, _p(cu, ip), T, hq, hkv, d, scale, int(causal),
+                                   _p(q, dp), _p(k, dp), _p(v, dp), n, _p(rows, ip), _p(heads, ip),
+                                   _p(o, dp), _p(lse, dp)), "attn_fwd_rows")
+    return o, lse
+
+
+def attn_bwd_rows(cu_seqlens, q, k, v, dout, scale: float, block: int, wblk, qrows, qheads,
+                  kvrows, kvheads, causal: bool = True):
+    """dQ at query rows (qrows, qheads) and dK, dV at KV rows (kvrows, kvheads)."""
+    cu = _i32(cu_seqlens)
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(dout)
+    T, hq, d = q.shape
+    hkv = k.shape[1]
+    nb = nblocks(cu, block)
+    if wblk is not None:
+        wb = _f64(wblk)
+        nbmax = wb.shape[2]
+        wptr = _p(wb, ctypes.c_double)
+    else:
+        nbmax = int(nb.max())
+        wptr = None
+    qrows, qheads, kvrows, kvheads = _i32(qrows), _i32(qheads), _i32(kvrows), _i32(kvheads)
+    dq = np.zeros((len(qrows), d))
+    dk = np.zeros((len(kvrows), d))
+    dv = np.zeros((len(kvrows), d))
+    dp, ip = ctypes.c_double, ctypes.c_int32
+    _check(lib().lfo_attn_bwd_rows(len(cu) - 1, _p(cu, ip), T, hq, hkv, d, scale, int(causal),
+                                   block, nbmax, _p(q, dp), _p(k, dp), _p(v, dp), _p(do, dp), wptr,
+                                   len(qrows), _p(qrows, ip), _p(qheads, ip), _p(dq, dp),
+                                   len(kvrows), _p(kvrows, ip), _p(kvheads, ip), _p(dk, dp),
+                                   _p(dv, dp)), "attn_bwd_rows")
     return dq, dk, dv

@@ -379,3 +379,168 @@ int lfo_attn_bwd(int nseq, const int32_t* cu, int T, int hq, int hkv, int d, dou
     }
     return LFO_OK;
 }
+
+/* ------------------------------------------------------------------------ */
+/* The same definitions evaluated only at chosen rows, for parity checks at    */
+/* sizes where the full oracle would take hours.  Nothing is reordered: each  */
+/* requested output is the same sum over the same rows as above.              */
+/* ------------------------------------------------------------------------ */
+
+static int segment_of(int nseq, const int32_t* cu, int t)
+{
+    int lo = 0, hi = nseq - 1;
+    while (lo < hi) {               /* last s with cu[s] <= t (skips empty segments) */
+        int mid = (lo + hi + 1) / 2;
+        if (cu[mid] <= t) lo = mid; else hi = mid - 1;
+    }
+    while (lo + 1 <= nseq - 1 && cu[lo + 1] <= t) ++lo;
+    return lo;
+}
+
+/* O and LSE of query rows (rows[r], heads[r]); o_out [nrows][d], lse_out [nrows]. */
+int lfo_attn_fwd_rows(int nseq, const int32_t* cu, int T, int hq, int hkv, int d, double scale,
+                      int causal, const double* q, const double* k, const double* v,
+                      int nrows, const int32_t* rows, const int32_t* heads,
+                      double* o_out, double* lse_out)
+{
+    if (check_desc(nseq, cu, T, hq, hkv, d)) return LFO_EINVAL;
+    int G = hq / hkv;
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < nrows; ++r) {
+        int t = rows[r], h = heads[r];
+        int s = segment_of(nseq, cu, t);
+        int len = cu[s + 1] - cu[s];
+        double* srow = (double*)malloc(sizeof(double) * (size_t)(len > 0 ? len : 1));
+        int n = row_scores(t, cu[s], cu[s + 1], causal, hq, hkv, d, scale, h, q, k, srow);
+        lse_out[r] = row_softmax(srow, n);
+        for (int c = 0; c < d; ++c) o_out[(size_t)r * d + c] = 0.0;
+        for (int i = 0; i < n; ++i) {
+            const double* vu = v + ((size_t)(cu[s] + i) * hkv + h / G) * d;
+            for (int c = 0; c < d; ++c) o_out[(size_t)r * d + c] += srow[i] * vu[c];
+        }
+        free(srow);
+    }
+    return LFO_OK;
+}
+
+/* Weighted backward at chosen rows: dq_out[r] = dQ[qrows[r], qheads[r], :];   */
+/* dk_out[r], dv_out[r] = dK, dV[kvrows[r], kvheads[r], :].  wblk as in         */
+/* lfo_attn_bwd (NULL = all ones).                                              */
+int lfo_attn_bwd_rows(int nseq, const int32_t* cu, int T, int hq, int hkv, int d, double scale,
+                      int causal, int block, int nbmax,
+                      const double* q, const double* k, const double* v, const double* dout,
+                      const double* wblk,
+                      int nq, const int32_t* qrows, const int32_t* qheads, double* dq_out,
+                      int nkv, const int32_t* kvrows, const int32_t* kvheads,
+                      double* dk_out, double* dv_out)
+{
+    if (check_desc(nseq, cu, T, hq, hkv, d) || block < 1) return LFO_EINVAL;
+    int G = hq / hkv;
+    /* dQ rows: each needs only its own softmax row */
+    #pragma omp parallel for schedule(dynamic, 1)
+    for (int r = 0; r < nq; ++r) {
+        int t = qrows[r], h = qheads[r], g = h / G;
+        int s = segment_of(nseq, cu, t), seg0 = cu[s];
+        int len = cu[s + 1] - seg0;
+        double* prow = (double*)malloc(sizeof(double) * (size_t)(len > 0 ? len : 1));
+        double* ot = (double*)calloc((size_t)d, sizeof(double));
+        double* dot_ = (double*)malloc(sizeof(double) * (size_t)d);
+        double wt = wblk ? wblk[((size_t)s * hq + h) * nbmax + (t - seg0) / block] : 1.0;
+        const double* dr = dout + ((size_t)t * hq + h) * d;
+        for (int c = 0; c < d; ++c) dot_[c] = wt * dr[c];
+        int n = row_scores(t, seg0, cu[s + 1], causal, hq, hkv, d, scale, h, q, k, prow);
+        (void)row_softmax(prow, n);
+        for (int i = 0; i < n; ++i) {
+            const double* vu = v + ((size_t)(seg0 + i) * hkv + g) * d;
+            for (int c = 0; c < d; ++c) ot[c] += prow[i] * vu[c];
+        }
+        double Dt = 0.0;
+        for (int c = 0; c < d; ++c) Dt += dot_[c] * ot[c];
+        double* out = dq_out + (size_t)r * d;
+        for (int c = 0; c < d; ++c) out[c] = 0.0;
+        for (int i = 0; i < n; ++i) {
+            const double* vu = v + ((size_t)(seg0 + i) * hkv + g) * d;
+            const double* ku = k + ((size_t)(seg0 + i) * hkv + g) * d;
+            double dP = 0.0;
+            for (int c = 0; c < d; ++c) dP += dot_[c] * vu[c];
+            double dS = prow[i] * (dP - Dt);
+            for (int c = 0; c < d; ++c) out[c] += scale * dS * ku[c];
+        }
+        free(prow); free(ot); free(dot_);
+    }
+    /* dK/dV rows: sum over every query row t of the group that sees key u.     */
+    /* Requested rows are handled per (segment, KV head): first LSE_t and D_t of */
+    /* every query row that can see one of them, then the per-pair terms.        */
+    char* done = (char*)calloc((size_t)(nkv > 0 ? nkv : 1), 1);
+    int* members = (int*)malloc(sizeof(int) * (size_t)(nkv > 0 ? nkv : 1));
+    for (int r0 = 0; r0 < nkv; ++r0) {
+        if (done[r0]) continue;
+        int g = kvheads[r0];
+        int s = segment_of(nseq, cu, kvrows[r0]), seg0 = cu[s], seg1 = cu[s + 1];
+        int nm = 0, umin = kvrows[r0];
+        for (int r = r0; r < nkv; ++r)
+            if (!done[r] && kvheads[r] == g && segment_of(nseq, cu, kvrows[r]) == s) {
+                done[r] = 1;
+                members[nm++] = r;
+                if (kvrows[r] < umin) umin = kvrows[r];
+            }
+        int t0 = causal ? umin : seg0;
+        int nt = seg1 - t0;
+        double* lse_t = (double*)malloc(sizeof(double) * (size_t)G * (nt > 0 ? nt : 1));
+        double* D_t = (double*)malloc(sizeof(double) * (size_t)G * (nt > 0 ? nt : 1));
+        #pragma omp parallel
+        {
+            double* prow = (double*)malloc(sizeof(double) * (size_t)(seg1 - seg0 > 0 ? seg1 - seg0 : 1));
+            double* ot = (double*)malloc(sizeof(double) * (size_t)d);
+            #pragma omp for collapse(2) schedule(dynamic, 4)
+            for (int hh = 0; hh < G; ++hh)
+                for (int it = 0; it < nt; ++it) {
+                    int h = g * G + hh, t = t0 + it;
+                    double wt = wblk ? wblk[((size_t)s * hq + h) * nbmax + (t - seg0) / block] : 1.0;
+                    int n = row_scores(t, seg0, seg1, causal, hq, hkv, d, scale, h, q, k, prow);
+                    double L = row_softmax(prow, n);
+                    for (int c = 0; c < d; ++c) ot[c] = 0.0;
+                    for (int i = 0; i < n; ++i) {
+                        const double* vi = v + ((size_t)(seg0 + i) * hkv + g) * d;
+                        for (int c = 0; c < d; ++c) ot[c] += prow[i] * vi[c];
+                    }
+                    const double* dr = dout + ((size_t)t * hq + h) * d;
+                    double Dt = 0.0;
+                    for (int c = 0; c < d; ++c) Dt += (wt * dr[c]) * ot[c];
+                    lse_t[(size_t)hh * nt + it] = L;
+                    D_t[(size_t)hh * nt + it] = Dt;
+                }
+            free(prow); free(ot);
+        }
+        #pragma omp parallel for schedule(dynamic, 1)
+        for (int mi = 0; mi < nm; ++mi) {
+            int r = members[mi], u = kvrows[r];
+            const double* vu = v + ((size_t)u * hkv + g) * d;
+            const double* ku = k + ((size_t)u * hkv + g) * d;
+            double* dk = dk_out + (size_t)r * d;
+            double* dv = dv_out + (size_t)r * d;
+            for (int c = 0; c < d; ++c) { dk[c] = 0.0; dv[c] = 0.0; }
+            for (int hh = 0; hh < G; ++hh) {
+                int h = g * G + hh;
+                for (int t = causal ? u : seg0; t < seg1; ++t) {
+                    double wt = wblk ? wblk[((size_t)s * hq + h) * nbmax + (t - seg0) / block] : 1.0;
+                    if (wt == 0.0) continue;     /* dO~_t = 0: the row adds exactly nothing */
+                    const double* qt = q + ((size_t)t * hq + h) * d;
+                    const double* dr = dout + ((size_t)t * hq + h) * d;
+                    double sc = 0.0, dP = 0.0;
+                    for (int c = 0; c < d; ++c) sc += qt[c] * ku[c];
+                    for (int c = 0; c < d; ++c) dP += (wt * dr[c]) * vu[c];
+                    double P = exp(scale * sc - lse_t[(size_t)hh * nt + (t - t0)]);
+                    double dS = P * (dP - D_t[(size_t)hh * nt + (t - t0)]);
+                    for (int c = 0; c < d; ++c) {
+                        dk[c] += scale * dS * qt[c];
+                        dv[c] += P * (wt * dr[c]);
+                    }
+                }
+            }
+        }
+        free(lse_t); free(D_t);
+    }
+    free(done); free(members);
+    return LFO_OK;
+}

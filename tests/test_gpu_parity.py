@@ -1,0 +1,258 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle on the
+same seeded bf16 inputs.
+
+Tolerances (fp32 accumulation of bf16 inputs on the GPU, fp64 in the oracle):
+keep masks, weights, tau and kept lists bit-exact given the same norm vector;
+block norms 1e-5 relative; O 1e-2 max-abs; LSE 1e-3 abs; dQ/dK/dV 1e-2
+relative Frobenius.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import block_sparse_attention_dense_b200 as lf
+import oracle
+import synthetic
+from _helpers import desc_for, nb_per_seq, rel_fro, run_step, to_dev
+
+pytestmark = pytest.mark.gpu
+
+O_TOL, LSE_TOL, GRAD_TOL, NORM_TOL = 1e-2, 1e-3, 1e-2, 1e-5
+
+# Small workloads the full oracle finishes in seconds; they span several tiles
+# and ragged tails.
+SMALL = [
+    synthetic.TINY,
+    synthetic.Workload("ragged_gqa", (700,), hq=4, hkv=2, d=128, block=128, sigma=1.5, delta=0.1),
+    synthetic.Workload("varlen_small", (1, 130, 0, 257, 64), hq=4, hkv=1, d=64, block=64,
+                       sigma=1.5, delta=0.2),
+    synthetic.Workload("mha_noncausal", (300, 200), hq=2, hkv=2, d=128, block=128, sigma=1.0,
+                       delta=0.05, causal=False),
+    synthetic.Workload("blk64_d128", (520,), hq=4, hkv=1, d=128, block=64, sigma=2.0, delta=0.3),
+]
+
+
+def _cpu(t):
+    return t.detach().float().cpu().numpy()
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_forward_matches_oracle(w):
+    inp = synthetic.make_inputs(w)
+    desc, dev, bufs = run_step(w, inp)
+    o_ref, lse_ref = oracle.attn_fwd(w.cu_seqlens(), inp["q"], inp["k"], inp["v"], w.scale, w.causal)
+    o = _cpu(bufs.o)
+    lse = _cpu(bufs.lse)
+    assert np.abs(o - o_ref).max() < O_TOL
+    assert np.abs(lse - lse_ref).max() < LSE_TOL
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_norms_and_rowdot_match_oracle(w):
+    inp = synthetic.make_inputs(w)
+    desc, dev, bufs = run_step(w, inp)
+    cu = w.cu_seqlens()
+    m_ref = oracle.block_norms(cu, inp["dout"], w.block, w.nbmax)
+    m = _cpu(bufs.norm)
+    assert np.all(np.abs(m - m_ref) <= NORM_TOL * np.maximum(m_ref, 1e-30))
+    # D from the same bf16 O the GPU stored
+    D_ref = oracle.rowdot(inp["dout"], bufs.o.cpu())
+    D = _cpu(bufs.D)
+    scale = np.sqrt(oracle.rowdot(inp["dout"], inp["dout"]) * oracle.rowdot(bufs.o.cpu(), bufs.o.cpu()))
+    assert np.all(np.abs(D - D_ref) <= 1e-5 * scale + 1e-30)
+
+
+def _select_case(nseq_lens, hq, block, sigma, seed):
+    w = synthetic.Workload("sel", tuple(nseq_lens), hq=hq, hkv=1 if hq % 2 else 2, d=64,
+                           block=block, sigma=sigma, delta=0.1)
+    nb = nb_per_seq(w)
+    m = synthetic.random_norms(w.nseq, hq, w.nbmax, nb, sigma, seed)
+    return w, nb, m
+
+
+@pytest.mark.parametrize("case", [
+    ((512,), 2, 64, 1.5),
+    ((32768,), 32, 128, 2.0),
+    (synthetic.VARLEN.seqlens, 32, 128, 1.5),
+    ((65536,), 4, 64, 2.0),
+    ((1, 100, 0, 5000), 8, 128, 0.5),
+], ids=["tiny", "headline", "varlen", "blk64_1024", "odd"])
+@pytest.mark.parametrize("delta", [0.0, 0.05, 0.1, 0.4, 0.95])
+def test_selection_bit_exact_given_norms(case, delta):
+    lens, hq, block, sigma = case
+    w, nb, m = _select_case(lens, hq, block, sigma, seed=hq + len(lens))
+    if sum(lens) == 0:
+        pytest.skip("empty")
+    m[0, 0, : min(3, nb[0])] = 0.0          # zero-norm blocks
+    desc = desc_for(w, torch.as_tensor(w.cu_seqlens()).cuda())
+    nbmax = w.nbmax
+    dummy = torch.zeros(w.total_tokens, hq, 64, dtype=torch.bfloat16, device="cuda")
+    norm = torch.as_tensor(m, device="cuda")
+    D = torch.empty(hq, w.total_tokens, device="cuda")
+    tau = torch.empty(w.nseq, hq, dtype=torch.float64, device="cuda")
+    wt = torch.empty(w.nseq, hq, nbmax, device="cuda")
+    keep = torch.empty(w.nseq, hq, nbmax, dtype=torch.uint8, device="cuda")
+    kidx = torch.empty(w.nseq, hq, nbmax, dtype=torch.int32, device="cuda")
+    kcnt = torch.empty(w.nseq, hq, dtype=torch.int32, device="cuda")
+    for seed, step in [(0, 0), (0x9E3779B97F4A7C15, 12345), (7, 2**32 + 3)]:
+        lf.lf_block_select(desc, dummy, dummy, delta, seed, step, lf.LF_SELECT_NORMS_GIVEN, norm, D,
+                           tau, wt, keep, kidx, kcnt)
+        lf.lf_check_device_error()
+        ref = oracle.select(m, nb, delta, seed, step)
+        np.testing.assert_array_equal(tau.cpu().numpy().view(np.uint64), ref["tau"].view(np.uint64))
+        np.testing.assert_array_equal(keep.cpu().numpy(), ref["keep"])
+        np.testing.assert_array_equal(wt.cpu().numpy().view(np.uint32), ref["w"].view(np.uint32))
+        np.testing.assert_array_equal(kcnt.cpu().numpy(), ref["kept_cnt"])
+        np.testing.assert_array_equal(kidx.cpu().numpy(), ref["kept_idx"])
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_backward_matches_oracle(w):
+    inp = synthetic.make_inputs(w)
+    desc, dev, bufs = run_step(w, inp, seed=3, step=1)
+    cu = w.cu_seqlens()
+    nb = nb_per_seq(w)
+    # the GPU's keep decisions equal the oracle's on the GPU's norms
+    sel = oracle.select(_cpu(bufs.norm), nb, w.delta, 3, 1)
+    np.testing.assert_array_equal(bufs.keep.cpu().numpy(), sel["keep"])
+    np.testing.assert_array_equal(bufs.w.cpu().numpy(), sel["w"])
+    dq_ref, dk_ref, dv_ref = oracle.attn_bwd(cu, inp["q"], inp["k"], inp["v"], inp["dout"],
+                                             w.scale, w.block, sel["w"].astype(np.float64),
+                                             w.causal)
+    assert rel_fro(_cpu(bufs.dq), dq_ref) < GRAD_TOL
+    assert rel_fro(_cpu(bufs.dk), dk_ref) < GRAD_TOL
+    assert rel_fro(_cpu(bufs.dv), dv_ref) < GRAD_TOL
+    # rows of dropped blocks get exactly zero dQ
+    dq = bufs.dq.cpu()
+    for s in range(w.nseq):
+        for h in range(w.hq):
+            for b in range(int(nb[s])):
+                if sel["keep"][s, h, b] == 0:
+                    r0 = cu[s] + b * w.block
+                    r1 = min(cu[s] + (b + 1) * w.block, cu[s + 1])
+                    assert torch.all(dq[r0:r1, h] == 0)
+
+
+@pytest.mark.parametrize("w", SMALL[:2], ids=lambda w: w.name)
+def test_delta_zero_is_the_dense_backward(w):
+    inp = synthetic.make_inputs(w)
+    desc, dev, bufs = run_step(w, inp, delta=0.0)
+    assert torch.all(bufs.keep.cpu()[:, :, : int(nb_per_seq(w).max())] == 1)
+    dq_ref, dk_ref, dv_ref = oracle.attn_bwd(w.cu_seqlens(), inp["q"], inp["k"], inp["v"],
+                                             inp["dout"], w.scale, w.block, None, w.causal)
+    assert rel_fro(_cpu(bufs.dq), dq_ref) < GRAD_TOL
+    assert rel_fro(_cpu(bufs.dk), dk_ref) < GRAD_TOL
+    assert rel_fro(_cpu(bufs.dv), dv_ref) < GRAD_TOL
+
+
+def test_heavy_budget_leaves_unreached_kv_tiles_zero():
+    w = synthetic.Workload("heavy", (1024,), hq=2, hkv=1, d=128, block=128, sigma=3.0, delta=0.95)
+    inp = synthetic.make_inputs(w)
+    desc, dev, bufs = run_step(w, inp, seed=1)
+    sel = oracle.select(_cpu(bufs.norm), nb_per_seq(w), w.delta, 1, 0)
+    dq_ref, dk_ref, dv_ref = oracle.attn_bwd(w.cu_seqlens(), inp["q"], inp["k"], inp["v"],
+                                             inp["dout"], w.scale, w.block,
+                                             sel["w"].astype(np.float64), True)
+    assert rel_fro(_cpu(bufs.dk), dk_ref) < GRAD_TOL
+    assert rel_fro(_cpu(bufs.dv), dv_ref) < GRAD_TOL
+    assert rel_fro(_cpu(bufs.dq), dq_ref) < GRAD_TOL
+    # a KV tile is reached only by kept blocks at or after it (causal)
+    kept = sel["keep"][0, :, :]
+    for j in range(8):
+        if not kept[:, j:].any():
+            assert torch.all(bufs.dk[j * 128:(j + 1) * 128] == 0)
+            assert torch.all(bufs.dv[j * 128:(j + 1) * 128] == 0)
+
+
+def test_same_seed_step_reproduces_and_steps_differ():
+    w = synthetic.GQA_MID.with_(seqlens=(2048,))
+    inp = synthetic.make_inputs(w)
+    _, _, b1 = run_step(w, inp, seed=5, step=9)
+    _, _, b2 = run_step(w, inp, seed=5, step=9)
+    _, _, b3 = run_step(w, inp, seed=5, step=10)
+    # masks, weights and the atomic-free dK/dV are bit-reproducible; dQ sums
+    # partial tiles with float atomics, so only its value is reproducible
+    assert torch.equal(b1.keep, b2.keep) and torch.equal(b1.w, b2.w)
+    assert torch.equal(b1.dk, b2.dk) and torch.equal(b1.dv, b2.dv) and torch.equal(b1.o, b2.o)
+    assert rel_fro(b1.dq.float().cpu(), b2.dq.float().cpu()) < 1e-5
+    assert not torch.equal(b1.keep, b3.keep)
+
+
+def test_empty_batch_is_a_noop():
+    cu = torch.zeros(2, dtype=torch.int32, device="cuda")
+    desc = lf.make_desc(cu, 0, 0, 2, 2, 64, 0.125, True, 64)
+    x = torch.zeros(16, dtype=torch.bfloat16, device="cuda")
+    f = torch.zeros(16, dtype=torch.float32, device="cuda")
+    lf.lf_attn_fwd(desc, x, x, x, x, f)
+    lf.lf_check_device_error()
+
+
+# ---------------------------------------------------------------------------
+# Full-size workloads, in the launch configuration the bench times: outputs the
+# oracle can compute one by one (sampled rows) plus properties at any size.
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("w", [synthetic.HEADLINE, synthetic.VARLEN], ids=lambda w: w.name)
+def test_full_size_sampled_parity(w):
+    inp = synthetic.make_inputs(w)
+    desc, dev, bufs = run_step(w, inp)
+    cu = w.cu_seqlens()
+    nb = nb_per_seq(w)
+    rng = np.random.default_rng(1)
+    # selection: bit-exact against the oracle on the GPU's norms
+    norms = _cpu(bufs.norm)
+    sel = oracle.select(norms, nb, w.delta, 0, 0)
+    np.testing.assert_array_equal(bufs.keep.cpu().numpy(), sel["keep"])
+    np.testing.assert_array_equal(bufs.kept_idx.cpu().numpy(), sel["kept_idx"])
+    np.testing.assert_array_equal(bufs.w.cpu().numpy().view(np.uint32), sel["w"].view(np.uint32))
+    # norms of sampled blocks
+    dout = inp["dout"]
+    for _ in range(16):
+        s = int(rng.integers(0, w.nseq))
+        h = int(rng.integers(0, w.hq))
+        b = int(rng.integers(0, nb[s]))
+        r0, r1 = cu[s] + b * w.block, min(cu[s] + (b + 1) * w.block, cu[s + 1])
+        ref = math.sqrt(float((dout[r0:r1, h].double() ** 2).sum()))
+        assert abs(norms[s, h, b] - ref) <= NORM_TOL * ref
+    # forward: sampled rows, including segment starts/ends and the last row
+    rows = list(rng.integers(0, w.total_tokens, size=24)) + [0, w.total_tokens - 1]
+    rows += [int(c) for c in cu[1:-1]] + [int(c) - 1 for c in cu[1:-1]]
+    rows = np.array(rows[:40], dtype=np.int32)
+    heads = rng.integers(0, w.hq, size=len(rows)).astype(np.int32)
+    o_ref, lse_ref = oracle.attn_fwd_rows(cu, inp["q"], inp["k"], inp["v"], w.scale, rows, heads)
+    o = _cpu(bufs.o)[rows, heads]
+    lse = _cpu(bufs.lse)[heads, rows]
+    assert np.abs(o - o_ref).max() < O_TOL
+    assert np.abs(lse - lse_ref).max() < LSE_TOL
+    # backward: dQ at sampled rows of kept blocks, zero at dropped blocks;
+    # dK/dV at the last KV tile of one segment (cheap for the row oracle)
+    wb = sel["w"].astype(np.float64)
+    kept_rows, kept_heads = [], []
+    dq = bufs.dq.cpu()
+    for _ in range(200):
+        s = int(rng.integers(0, w.nseq))
+        h = int(rng.integers(0, w.hq))
+        b = int(rng.integers(0, nb[s]))
+        t = int(cu[s] + b * w.block + rng.integers(0, min(w.block, cu[s + 1] - cu[s] - b * w.block)))
+        if sel["keep"][s, h, b]:
+            if len(kept_rows) < 24:
+                kept_rows.append(t)
+                kept_heads.append(h)
+        else:
+            assert torch.all(dq[t, h] == 0)
+    s_last = w.nseq - 1
+    u0 = max(int(cu[s_last + 1]) - 128, int(cu[s_last]))
+    kv_rows = np.arange(u0, int(cu[s_last + 1]), 8, dtype=np.int32)
+    kv_heads = (np.arange(len(kv_rows)) % w.hkv).astype(np.int32)
+    dq_ref, dk_ref, dv_ref = oracle.attn_bwd_rows(cu, inp["q"], inp["k"], inp["v"], dout, w.scale,
+                                                  w.block, wb, kept_rows, kept_heads, kv_rows,
+                                                  kv_heads)
+    assert rel_fro(_cpu(bufs.dq)[kept_rows, kept_heads], dq_ref) < GRAD_TOL
+    dk = _cpu(bufs.dk)[kv_rows, kv_heads]
+    dv = _cpu(bufs.dv)[kv_rows, kv_heads]
+    if np.linalg.norm(dk_ref) > 0:
+        assert rel_fro(dk, dk_ref) < GRAD_TOL
+        assert rel_fro(dv, dv_ref) < GRAD_TOL
+    else:
+        assert np.all(dk == 0) and np.all(dv == 0)

@@ -173,3 +173,32 @@ def test_block_norms_and_rowdot_match_numpy():
                 assert abs(m[s, h, i] - ref) <= 1e-13 * max(ref, 1.0)
     D = oracle.rowdot(do, o)
     np.testing.assert_allclose(D, np.einsum("thd,thd->ht", d, o.numpy()), rtol=1e-13, atol=1e-13)
+
+
+@pytest.mark.parametrize("causal", [True, False])
+def test_row_sampled_oracle_equals_full_oracle(causal):
+    # The row-sampled evaluation (used for parity at full size) must agree with
+    # the full oracle at those rows, including empty segments and GQA.
+    cu = np.array([0, 40, 40, 131, 200], dtype=np.int32)
+    T, hq, hkv, d, block = 200, 4, 2, 8, 16
+    q, k, v = _rand((T, hq, d), 71), _rand((T, hkv, d), 72), _rand((T, hkv, d), 73)
+    do = _rand((T, hq, d), 74)
+    nbmax = int(oracle.nblocks(cu, block).max())
+    w = np.random.default_rng(2).uniform(0.0, 3.0, size=(4, hq, nbmax))
+    w[:, :, 1] = 0.0
+    scale = 0.35
+    o, lse = oracle.attn_fwd(cu, q, k, v, scale, causal)
+    dq, dk, dv = oracle.attn_bwd(cu, q, k, v, do, scale, block, w, causal)
+    rng = np.random.default_rng(4)
+    rows = rng.integers(0, T, size=25)
+    heads = rng.integers(0, hq, size=25)
+    o_r, lse_r = oracle.attn_fwd_rows(cu, q, k, v, scale, rows, heads, causal)
+    np.testing.assert_allclose(o_r, o[rows, heads], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse_r, lse[heads, rows], rtol=1e-12, atol=1e-13)
+    kvr = rng.integers(0, T, size=20)
+    kvh = rng.integers(0, hkv, size=20)
+    dq_r, dk_r, dv_r = oracle.attn_bwd_rows(cu, q, k, v, do, scale, block, w, rows, heads,
+                                            kvr, kvh, causal)
+    np.testing.assert_allclose(dq_r, dq[rows, heads], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dk_r, dk[kvr, kvh], rtol=1e-10, atol=1e-12)
+    np.testing.assert_allclose(dv_r, dv[kvr, kvh], rtol=1e-10, atol=1e-12)
