@@ -1,0 +1,370 @@
+"""LazyFlash attention step benchmark (forward + selection + sparse backward).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl lazyflash|reference]
+                    [--workload headline|varlen|long|gqa_mid|tiny] [--delta D]
+
+One step = the whole hot path over one batch: lf_attn_fwd, lf_block_select and
+lf_attn_bwd on the workload's synthetic bf16 inputs (a Qwen3-8B-shaped layer:
+Hq=32, Hkv=8, d=128; N=32768 tokens, delta=0.1 by default).  Inputs stay
+resident in HBM for `value`; `e2e` repeats the step through the same API with
+host (pinned) inputs copied in and the results (O, LSE, dQ, dK, dV) copied out
+inside the timed region.  Every input tensor is larger than L2 (126 MB), so no
+explicit flush is needed between steps.
+
+Under torchrun each rank runs an independent replica (the path has no data
+exchange): `value` = all ranks' FLOPs / the slowest rank's time.
+
+`--impl reference` times the CPU oracle (fp64 C, OpenMP) on a bounded sample of
+the same workload, on rank 0 only.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synthetic  # noqa: E402
+
+TILE = 128
+
+
+def _load_json(path):
+    try:
+        with open(path) as f:
+            return json.load(f)
+    except Exception:
+        return None
+
+
+def tile_flops(w: synthetic.Workload, keep=None):
+    """Tile-level FLOPs: forward (all tiles), backward dense-equivalent and
+    backward executed (query tiles holding a kept block).  ntile(i) = KV tiles
+    a 128-row query tile i meets: i + 1 causal, all tiles of the segment
+    otherwise.  Forward: 4*128*128*d per (query tile, KV tile); backward: 10*."""
+    unit = TILE * TILE * w.d
+    fwd = bwd_dense = bwd_exec = 0
+    per = TILE // w.block
+    for s, L in enumerate(w.seqlens):
+        nt = (L + TILE - 1) // TILE
+        for i in range(nt):
+            n_kv = (i + 1) if w.causal else nt
+            fwd += w.hq * n_kv * 4 * unit
+            bwd_dense += w.hq * n_kv * 10 * unit
+            if keep is not None:
+                b0 = i * per
+                kept_heads = keep[s, :, b0:b0 + per].any(axis=1).sum()
+                bwd_exec += int(kept_heads) * n_kv * 10 * unit
+    return fwd, bwd_dense, bwd_exec
+
+
+# ---------------------------------------------------------------------------
+# clocks during the timed region
+# ---------------------------------------------------------------------------
+_CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+                 "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+                 "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+
+class ClockSampler:
+    def __init__(self, device_index: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        uuid = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+        except Exception:
+            pass
+        sel = ["-i", uuid] if uuid else []
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "--query-gpu=" + _CLOCK_FIELDS,
+                                       "--format=csv,noheader,nounits", "-lms", "100", *sel],
+                                      stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except Exception:
+            self.p.kill()
+        self.f.flush()
+        self.f.seek(0)
+        rows = [r.split(",") for r in self.f.read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle sample (the cpu_baseline and the reference arm)
+# ---------------------------------------------------------------------------
+def oracle_sample(w: synthetic.Workload, inp, prefix: int, seed=0, step=0):
+    """The oracle's forward, selection and weighted backward on the first
+    `prefix` tokens of segment 0 (a causal prefix is itself a complete problem),
+    all heads.  Returns (seconds, executed tile FLOPs of the sample, threads)."""
+    import oracle
+    ws = w.with_(seqlens=(prefix,))
+    sl = slice(0, prefix)
+    q, k, v, do = inp["q"][sl], inp["k"][sl], inp["v"][sl], inp["dout"][sl]
+    cu = ws.cu_seqlens()
+    oracle.lib()
+    t0 = time.perf_counter()
+    o, lse = oracle.attn_fwd(cu, q, k, v, ws.scale, ws.causal)
+    m = oracle.block_norms(cu, do, ws.block)
+    sel = oracle.select(m, oracle.nblocks(cu, ws.block), ws.delta, seed, step)
+    oracle.attn_bwd(cu, q, k, v, do, ws.scale, ws.block, sel["w"].astype(np.float64), ws.causal)
+    dt = time.perf_counter() - t0
+    f, _, b = tile_flops(ws, sel["keep"])
+    threads = int(os.environ.get("OMP_NUM_THREADS", len(os.sched_getaffinity(0))))
+    return dt, f + b, threads
+
+
+def run_reference(args, w, rank):
+    if rank != 0:
+        return
+    prefix = min(args.ref_prefix, w.seqlens[0])
+    inp = synthetic.make_inputs(w, rows=prefix) if w.nseq == 1 else synthetic.make_inputs(w)
+    for _ in range(args.warmup):
+        oracle_sample(w, inp, prefix)
+    tot_t = tot_f = 0.0
+    threads = 1
+    for _ in range(args.steps):
+        dt, fl, threads = oracle_sample(w, inp, prefix)
+        tot_t += dt
+        tot_f += fl
+    val = tot_f / tot_t / 1e12
+    sample = ("oracle fwd+select+bwd on the first %d tokens of the %s workload, all %d heads "
+              "(a causal prefix is a complete sub-problem)" % (prefix, w.name, w.hq))
+    line = {
+        "impl": "reference", "metric": args.metric, "value": val, "unit": "TFLOP/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_of(w, args),
+        "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def config_of(w, args):
+    return {"workload": w.name, "seqlens": list(w.seqlens) if w.nseq <= 16 else "%d segments" % w.nseq,
+            "total_tokens": w.total_tokens, "hq": w.hq, "hkv": w.hkv, "d": w.d, "block": w.block,
+            "causal": w.causal, "delta": w.delta, "dO_block_scale": "LogNormal(0,%g)" % w.sigma,
+            "seed": 0, "step": 0,
+            "l2": "no flush: every input tensor (>= 64 MiB x4 heads) exceeds L2 per step",
+            "parallelism": "replicas" if args.gpus > 1 else "single"}
+
+
+# ---------------------------------------------------------------------------
+# LazyFlash arm
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="lazyflash", choices=["lazyflash", "reference"])
+    ap.add_argument("--workload", default="headline", choices=sorted(synthetic.WORKLOADS))
+    ap.add_argument("--delta", type=float, default=None)
+    ap.add_argument("--cpu-prefix", type=int, default=2048,
+                    help="tokens of the oracle sample timed for cpu_baseline")
+    ap.add_argument("--ref-prefix", type=int, default=1024,
+                    help="tokens of the oracle sample timed per step by --impl reference")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.metric = "LazyFlash attn bwd ms & executed TFLOP/s at N=32K, Hq32/Hkv8 d128, delta=0.1"
+    w = synthetic.WORKLOADS[args.workload]
+    if args.delta is not None:
+        w = w.with_(delta=args.delta)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local))
+    if args.impl == "reference":
+        run_reference(args, w, rank)
+        if dist is not None:
+            dist.destroy_process_group()
+        return
+
+    import block_sparse_attention_dense_b200 as lf
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+
+    inp = synthetic.make_inputs(w)
+    host = {k: v.pin_memory() for k, v in inp.items() if k != "cu_seqlens"}
+    d_in = {k: v.to(dev) for k, v in host.items()}
+    cu = inp["cu_seqlens"].to(dev)
+    desc = lf.make_desc(cu, w.max_seqlen, w.total_tokens, w.hq, w.hkv, w.d, w.scale, w.causal,
+                        w.block)
+    bufs = lf.Buffers(desc, device=dev)
+
+    def step():
+        lf.lf_attn_fwd(desc, d_in["q"], d_in["k"], d_in["v"], bufs.o, bufs.lse)
+        lf.lf_block_select(desc, d_in["dout"], bufs.o, w.delta, 0, 0, 0, bufs.norm, bufs.D,
+                           bufs.tau, bufs.w, bufs.keep, bufs.kept_idx, bufs.kept_cnt)
+        lf.lf_attn_bwd(desc, d_in["q"], d_in["k"], d_in["v"], bufs.o, bufs.lse, d_in["dout"],
+                       bufs.D, bufs.w, bufs.kept_idx, bufs.kept_cnt, bufs.dq, bufs.dk, bufs.dv,
+                       bufs.ws)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    lf.lf_check_device_error()
+    torch.cuda.synchronize()
+    keep = bufs.keep.cpu().numpy()
+    fwd_fl, bwd_dense_fl, bwd_exec_fl = tile_flops(w, keep)
+
+    # ---- device-timed steps, inputs resident; per-phase events on the launching stream
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    start = torch.cuda.Event(enable_timing=True)
+    end = torch.cuda.Event(enable_timing=True)
+    start.record(stream)
+    for i in range(K):
+        e = ev[i]
+        e[0].record(stream)
+        lf.lf_attn_fwd(desc, d_in["q"], d_in["k"], d_in["v"], bufs.o, bufs.lse)
+        e[1].record(stream)
+        lf.lf_block_select(desc, d_in["dout"], bufs.o, w.delta, 0, 0, 0, bufs.norm, bufs.D,
+                           bufs.tau, bufs.w, bufs.keep, bufs.kept_idx, bufs.kept_cnt)
+        e[2].record(stream)
+        lf.lf_attn_bwd(desc, d_in["q"], d_in["k"], d_in["v"], bufs.o, bufs.lse, d_in["dout"],
+                       bufs.D, bufs.w, bufs.kept_idx, bufs.kept_cnt, bufs.dq, bufs.dk, bufs.dv,
+                       bufs.ws)
+        e[3].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    clk = clocks.stop()
+    total_ms = start.elapsed_time(end)
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
+    sel_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
+    bwd_ms = sum(e[2].elapsed_time(e[3]) for e in ev) / K
+    lf.lf_check_device_error()
+
+    # ---- end to end through the API: host inputs in, results out, every step
+    h_out = {"o": torch.empty_like(bufs.o, device="cpu").pin_memory(),
+             "lse": torch.empty_like(bufs.lse, device="cpu").pin_memory(),
+             "dq": torch.empty_like(bufs.dq, device="cpu").pin_memory(),
+             "dk": torch.empty_like(bufs.dk, device="cpu").pin_memory(),
+             "dv": torch.empty_like(bufs.dv, device="cpu").pin_memory()}
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = sum(t.numel() * t.element_size() for t in h_out.values())
+    Ke = max(3, min(K, 10))
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e2s = torch.cuda.Event(enable_timing=True)
+    e2e = torch.cuda.Event(enable_timing=True)
+    e2s.record(stream)
+    for _ in range(Ke):
+        for k_, t in host.items():
+            d_in[k_].copy_(t, non_blocking=True)
+        step()
+        for k_, t in h_out.items():
+            t.copy_(getattr(bufs, k_), non_blocking=True)
+    e2e.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e2s.elapsed_time(e2e)
+
+    # ---- max over ranks
+    if dist is not None:
+        tt = torch.tensor([total_ms, e2e_ms], device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        total_ms, e2e_ms = float(tt[0]), float(tt[1])
+
+    n = world
+    step_fl = fwd_fl + bwd_exec_fl
+    value = n * K * step_fl / (total_ms * 1e-3) / 1e12
+    e2e_val = n * Ke * step_fl / (e2e_ms * 1e-3) / 1e12
+    peaks = _load_json(os.path.join(ROOT, "MEASURED_PEAKS.json"))
+    if peaks:
+        peak, peak_src = float(peaks["bf16_tflops_sustained"]), "measured (sustained)"
+    else:
+        peak, peak_src = 1400.0, "fallback (sustained)"
+    fwd_tf = fwd_fl / (fwd_ms * 1e-3) / 1e12
+    bwd_tf = bwd_exec_fl / (bwd_ms * 1e-3) / 1e12
+    dom = "attn_fwd_kernel" if fwd_ms >= bwd_ms else "attn_bwd (memset + attn_bwd_kernel + dq_convert)"
+    achieved = fwd_tf if fwd_ms >= bwd_ms else bwd_tf
+    traffic = _load_json(os.path.join(ROOT, "profiles", "traffic.json")) or {}
+    line = {
+        "metric": args.metric, "value": value, "unit": "TFLOP/s", "n_gpus": n, "steps": K,
+        "warmup": max(3, args.warmup), "ms_per_step": total_ms / K, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": config_of(w, args),
+        "phases_ms": {"fwd": fwd_ms, "select": sel_ms, "bwd": bwd_ms},
+        "bwd_ms": bwd_ms, "bwd_tflops_executed": bwd_tf,
+        "bwd_tflops_dense_equiv": bwd_dense_fl / (bwd_ms * 1e-3) / 1e12,
+        "fwd_tflops": fwd_tf,
+        "flops_per_step": {"fwd": fwd_fl, "bwd_executed": bwd_exec_fl, "bwd_dense": bwd_dense_fl},
+        "kept_fraction": float(keep.astype(bool).sum() / max(1, int(sum(
+            (L + w.block - 1) // w.block for L in w.seqlens)) * w.hq)),
+        "bwd_executed_fraction": bwd_exec_fl / bwd_dense_fl,
+        "roofline": {"bound": "tensor", "kernel": dom, "achieved": achieved, "peak": peak,
+                     "peak_source": peak_src, "unit": "TFLOP/s", "frac": achieved / peak,
+                     "traffic": traffic.get(dom.split()[0])},
+        "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / Ke, "steps": Ke},
+        "gpu_launches": 5 * K,
+        "clocks": clk,
+    }
+    if rank == 0 and n == 1 and not args.no_cpu_baseline:
+        dt, fl, threads = oracle_sample(w, inp, min(args.cpu_prefix, w.seqlens[0]))
+        line["cpu_baseline"] = {
+            "value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
+            "seconds": dt,
+            "sample": "oracle fwd+select+bwd on the first %d tokens of the %s workload, all %d "
+                      "heads" % (min(args.cpu_prefix, w.seqlens[0]), w.name, w.hq)}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

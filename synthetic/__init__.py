@@ -7,10 +7,11 @@ Both the CUDA path and the CPU oracle receive the arrays built here.
 Recipe (the article's LongAlign/Qwen3-8B training data is not available, so
 seeded tensors with the same attention shapes stand in for it):
 
-* ``numpy.random.Generator(PCG64(seed))`` draws, in this order, Q, K, V and a
-  base dO as float32 standard normals, then one LogNormal(0, sigma) scale per
-  (segment, query head, block of ``block`` rows); every dO row of a block is
-  multiplied by that block's scale.  The skewed per-block scale reproduces the
+* ``numpy.random.SeedSequence(seed)`` spawns five independent PCG64 streams:
+  Q, K, V and a base dO as float32 standard normals (row-major, so the first
+  rows of a tensor never depend on how many rows follow), and one
+  LogNormal(0, sigma) scale per (segment, query head, block of ``block``
+  rows); every dO row of a block is multiplied by that block's scale.  The skewed per-block scale reproduces the
   uneven spread of output-gradient mass across query blocks that the LazyFlash
   article builds on ("Le passage arrière fait deux fois le travail du passage
   avant").
@@ -106,18 +107,25 @@ def _bf16(a: np.ndarray) -> torch.Tensor:
     return torch.from_numpy(a).to(torch.bfloat16)
 
 
-def make_inputs(w: Workload, seed: Optional[int] = None) -> dict:
-    """Host bf16 tensors q, k, v, dout (THD) plus cu_seqlens for workload ``w``."""
+def make_inputs(w: Workload, seed: Optional[int] = None, rows: Optional[int] = None) -> dict:
+    """Host bf16 tensors q, k, v, dout (THD) plus cu_seqlens for workload ``w``.
+
+    ``rows`` < T returns only the first ``rows`` tokens (identical to the same
+    rows of the full draw) with a single segment; it requires ``w`` to have one
+    segment, so that a causal prefix is itself a complete problem."""
     seed = w.seed if seed is None else seed
-    rng = np.random.Generator(np.random.PCG64(seed))
-    T = w.total_tokens
-    q = rng.standard_normal((T, w.hq, w.d), dtype=np.float32)
-    k = rng.standard_normal((T, w.hkv, w.d), dtype=np.float32)
-    v = rng.standard_normal((T, w.hkv, w.d), dtype=np.float32)
-    do = rng.standard_normal((T, w.hq, w.d), dtype=np.float32)
-    scales = rng.lognormal(0.0, w.sigma, size=(w.nseq, w.hq, w.nbmax)).astype(np.float32)
-    cu = w.cu_seqlens()
-    for s in range(w.nseq):
+    streams = [np.random.Generator(np.random.PCG64(c))
+               for c in np.random.SeedSequence(seed).spawn(5)]
+    T = w.total_tokens if rows is None else int(rows)
+    if rows is not None and (w.nseq != 1 or not 0 < T <= w.total_tokens):
+        raise ValueError("a prefix needs a single-segment workload and 0 < rows <= T")
+    q = streams[0].standard_normal((T, w.hq, w.d), dtype=np.float32)
+    k = streams[1].standard_normal((T, w.hkv, w.d), dtype=np.float32)
+    v = streams[2].standard_normal((T, w.hkv, w.d), dtype=np.float32)
+    do = streams[3].standard_normal((T, w.hq, w.d), dtype=np.float32)
+    scales = streams[4].lognormal(0.0, w.sigma, size=(w.nseq, w.hq, w.nbmax)).astype(np.float32)
+    cu = w.cu_seqlens() if rows is None else np.array([0, T], dtype=np.int32)
+    for s in range(len(cu) - 1):
         a, b = int(cu[s]), int(cu[s + 1])
         nb = (b - a + w.block - 1) // w.block
         for i in range(nb):

@@ -77,3 +77,13 @@ def test_gqa_mapping_is_consecutive_groups():
     np.testing.assert_array_equal(o[:, 0], o[:, 1])
     np.testing.assert_array_equal(o[:, 2], o[:, 3])
     assert np.abs(o[:, 0] - o[:, 2]).max() > 1e-3
+
+
+def test_synthetic_prefix_equals_full_draw():
+    import synthetic
+    w = synthetic.TINY.with_(seqlens=(300,))
+    full = synthetic.make_inputs(w)
+    pre = synthetic.make_inputs(w, rows=130)
+    for k in ("q", "k", "v", "dout"):
+        assert torch.equal(full[k][:130], pre[k])
+    assert list(pre["cu_seqlens"]) == [0, 130]
