@@ -187,3 +187,16 @@ def lazyflash_step(desc, q, k, v, dout, delta, seed, step, bufs: Buffers, flags=
                     bufs.w, bufs.keep, bufs.kept_idx, bufs.kept_cnt, stream=stream)
     lf_attn_bwd(desc, q, k, v, bufs.o, bufs.lse, dout, bufs.D, bufs.w, bufs.kept_idx,
                 bufs.kept_cnt, bufs.dq, bufs.dk, bufs.dv, bufs.ws, stream=stream)
+
+
+def lf_attn_bwd_static_ws(desc, q, k, v, o, lse, dout, D, block_weight, kept_idx, kept_cnt, dq,
+                          dk, dv, stream=None):
+    """lf_attn_bwd with the library's static scratch array instead of a caller
+    workspace (for callers that cannot allocate; see include/lazyflash.h)."""
+    L = _load()
+    fn = L.lf_attn_bwd_static_ws
+    fn.argtypes = [ctypes.POINTER(lf_attn_desc)] + [ctypes.c_void_p] * 14
+    fn.restype = ctypes.c_int
+    _check(fn(ctypes.byref(desc), _ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(dout),
+              _ptr(D), _ptr(block_weight), _ptr(kept_idx), _ptr(kept_cnt), _ptr(dq), _ptr(dk),
+              _ptr(dv), _stream(stream)), "lf_attn_bwd_static_ws")

@@ -169,6 +169,34 @@ lf_status launch_bwd(const lf_attn_desc* d, const void* q, const void* k, const 
 
 }  // namespace
 
+// Scratch of lf_attn_bwd_static_ws: one array per device, loaded with the
+// library and kept until the process exits.  Host code must not use this name
+// as a device address (it names a host-side stand-in); the device address comes
+// from cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char lf_static_ws[LF_STATIC_WS_BYTES];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_static_ws_mutex;
+void* g_static_ws_ptr[kMaxDevices] = {};
+
+// Device address of lf_static_ws on the current device (looked up once per device).
+lf_status static_ws_address(void** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LF_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+    if (!g_static_ws_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, lf_static_ws) != cudaSuccess || !p) return LF_ERR_CUDA;
+        g_static_ws_ptr[dev] = p;
+    }
+    *out = g_static_ws_ptr[dev];
+    return LF_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* lf_status_string(lf_status s) {
@@ -278,6 +306,46 @@ lf_status lf_attn_bwd(const lf_attn_desc* desc, const void* q, const void* k, co
         if (st != LF_OK) return st;
         Dv = Dw;
     }
+    return desc->d == 128 ? launch_bwd<128>(desc, q, k, v, lse, dout, Dv, block_weight, kept_idx,
+                                            kept_cnt, dq, dk, dv, dq_acc, s)
+                          : launch_bwd<64>(desc, q, k, v, lse, dout, Dv, block_weight, kept_idx,
+                                           kept_cnt, dq, dk, dv, dq_acc, s);
+}
+
+lf_status lf_attn_bwd_static_ws(const lf_attn_desc* desc, const void* q, const void* k,
+                                const void* v, const void* o, const float* lse, const void* dout,
+                                const float* D, const float* block_weight,
+                                const int32_t* kept_idx, const int32_t* kept_cnt, void* dq,
+                                void* dk, void* dv, lf_stream_t stream) {
+    lf_status st = check_desc(desc);
+    if (st != LF_OK) return st;
+    if (!q || !k || !v || !lse || !dout || !block_weight || !kept_idx || !kept_cnt || !dq ||
+        !dk || !dv)
+        return LF_ERR_INVALID_ARG;
+    if (!D && !o) return LF_ERR_INVALID_ARG;
+    const void* ptrs[] = {q, k, v, lse, dout, block_weight, kept_idx, kept_cnt, dq, dk, dv};
+    for (const void* p : ptrs)
+        if (!aligned16(p)) return LF_ERR_INVALID_ARG;
+    if ((o && !aligned16(o)) || (D && !aligned16(D))) return LF_ERR_INVALID_ARG;
+    const size_t need = bwd_ws_bytes(desc, D == nullptr);
+    if (need > LF_STATIC_WS_BYTES) return LF_ERR_WORKSPACE;
+    if (desc->total_tokens == 0 || desc->max_seqlen == 0) return LF_OK;
+    void* ws = nullptr;
+    st = static_ws_address(&ws);
+    if (st != LF_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    float* dq_acc = static_cast<float*>(ws);
+    const float* Dv = D;
+    if (!Dv) {
+        const size_t acc = ((size_t)desc->total_tokens * desc->hq * desc->d * sizeof(float) + 255) &
+                           ~size_t(255);
+        float* Dw = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + acc);
+        st = desc->d == 128 ? launch_norms<128>(desc, dout, o, nullptr, Dw, 0, s)
+                            : launch_norms<64>(desc, dout, o, nullptr, Dw, 0, s);
+        if (st != LF_OK) return st;
+        Dv = Dw;
+    }
+    // launch_bwd clears the accumulator (cudaMemsetAsync) before the kernel
     return desc->d == 128 ? launch_bwd<128>(desc, q, k, v, lse, dout, Dv, block_weight, kept_idx,
                                             kept_cnt, dq, dk, dv, dq_acc, s)
                           : launch_bwd<64>(desc, q, k, v, lse, dout, Dv, block_weight, kept_idx,

@@ -132,6 +132,37 @@ lf_status lf_attn_bwd(const lf_attn_desc* desc, const void* q, const void* k, co
                       const int32_t* kept_cnt, void* dq, void* dk, void* dv,
                       void* ws, size_t ws_bytes, lf_stream_t stream);
 
+/* Capacity of the library's static scratch array used by lf_attn_bwd_static_ws. */
+#define LF_STATIC_WS_BYTES ((size_t)32 << 20)
+
+/* lf_attn_bwd without a workspace argument and without any allocation.
+ * The paper has no counterpart to this entry point; it exists for callers that
+ * cannot allocate device memory on the library's behalf: custom-op plugin
+ * interfaces that hand an operator only its inputs and outputs, and runtimes
+ * that plan all device memory ahead of time or forbid cudaMalloc/cudaFree while
+ * they run (those calls synchronize the device and are not allowed inside a
+ * stream capture).
+ *   Arguments and results are those of lf_attn_bwd.  The scratch (the fp32 dQ
+ *   accumulator, plus D when D is NULL) lives in one file-scope device array of
+ *   LF_STATIC_WS_BYTES bytes that every GPU loading the library holds until the
+ *   process exits.  A problem whose scratch exceeds it, i.e.
+ *   4 * total_tokens * hq * d bytes (rounded up to 256), plus
+ *   4 * total_tokens * hq when D is NULL, returns LF_ERR_WORKSPACE before
+ *   anything is launched.
+ *   The first call on a device looks up the array's device address
+ *   (cudaGetSymbolAddress, with that device current); make that first call
+ *   before any stream capture.  The call never calls cudaMalloc, cudaFree or an
+ *   allocating library routine; the accumulator is cleared at the start of
+ *   every call.
+ *   All calls on a device share the one array and it keeps the last call's
+ *   contents: calls that may overlap on the GPU (different streams, or host
+ *   threads without ordering) race on it and produce wrong dQ. */
+lf_status lf_attn_bwd_static_ws(const lf_attn_desc* desc, const void* q, const void* k,
+                                const void* v, const void* o, const float* lse, const void* dout,
+                                const float* D, const float* block_weight,
+                                const int32_t* kept_idx, const int32_t* kept_cnt, void* dq,
+                                void* dk, void* dv, lf_stream_t stream);
+
 /* Waits for `stream`, then reads and clears the device watchdog flag.
  * LF_ERR_TIMEOUT if a kernel gave up a bounded wait since the last check,
  * LF_ERR_CUDA if the stream reported an error, else LF_OK. */
