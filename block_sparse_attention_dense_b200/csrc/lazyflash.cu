@@ -157,7 +157,7 @@ lf_status launch_bwd(const lf_attn_desc* d, const void* q, const void* k, const 
     if (cudaFuncSetAttribute(lf::attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem) != cudaSuccess)
         return LF_ERR_CUDA;
-    dim3 grid(d->hkv, ntiles_of(d), d->nseq);
+    dim3 grid(ntiles_of(d), d->hkv, d->nseq);
     lf::attn_bwd_kernel<D><<<grid, lf::kBwdThreads, smem, st>>>(mq, mk, mv, mdo, p);
     if (launch_status() != LF_OK) return LF_ERR_CUDA;
     const size_t n8 = nacc / 8;

@@ -6,18 +6,26 @@
 //
 // One CTA owns a 128-row KV tile j of one KV head g of one segment and walks,
 // for every query head of g's group, the kept query tiles t (t >= j when
-// causal) from the compacted kept-block lists.  Per (t, j) pair:
-//   tcgen05:  S^T  = K_j Q_t^T           (TMEM, 128 KV lanes x 128 q cols)
-//             dP^T = V_j dO_t^T          (TMEM)
-//   4 warps:  thread r owns KV row r:  P = exp2(S * scale*log2e - LSE*log2e),
-//             dS = P (dP - D), both times the column's block weight, rounded
-//             to bf16 into shared memory (K-major over q)
-//   tcgen05:  dV_j += P^T dO_t, dK_j += dS^T Q_t   (TMEM, accumulated over the
-//             whole walk: no atomics for dK/dV), dQ_t(partial) = dS K_j (TMEM)
-//   4 warps:  thread r now owns query row r of the partial dQ and adds it into
-//             the fp32 dQ accumulator (vector atomics).
-// The epilogue writes dK (times softmax_scale) and dV as bf16; a KV tile that
-// no kept block reaches gets zeros.
+// causal) from the compacted kept-block lists.  Each 128-row query tile is
+// handled as two 64-column halves so that the element-wise work on one half
+// overlaps the tensor-core work on the other.  Per half:
+//   tcgen05 (SS): S^T  = K_j Q_h^T,  dP^T = V_j dO_h^T        (TMEM, fp32)
+//   element-wise: P = exp2(S*scale*log2e - LSE*log2e), dS = P (dP - D), both
+//                 times the block weight; P^T and dS^T rounded to bf16 back
+//                 into TMEM (over S^T / dP^T) and dS^T into shared memory
+//   tcgen05 (TS): dV_j += P^T dO_h, dK_j += dS^T Q_h   (A from TMEM; dK/dV
+//                 accumulate in TMEM over the whole walk: no atomics)
+//   tcgen05 (SS): dQ_h^T = K_j^T dS^T_h                  (TMEM, lanes = d)
+//   dQ drain:     lane d adds column q of dQ_h^T into the fp32 accumulator;
+//                 a warp's 32 lanes hit 32 consecutive floats of one row.
+// Roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer, warps 4-7
+// element-wise + epilogue (thread = KV row = TMEM lane), warps 8-11 dQ drain
+// (thread = head-dim index = TMEM lane).  The epilogue writes dK (times
+// softmax_scale) and dV as bf16; a KV tile that no kept block reaches gets 0.
+//
+// Tensor memory (512 columns): dV [0,128) dK [128,256); half 0: S^T/P^T/dQ^T
+// [256,320), dP^T/dS^T [320,384); half 1: [384,448), [448,512).  Reuse of a
+// region by a later MMA relies on tcgen05.mma executing in issue order.
 #pragma once
 
 #include "lf_device.cuh"
@@ -43,22 +51,29 @@ template <int D>
 struct BwdSmem {
     static constexpr int kPanels = D / 64;
     static constexpr uint32_t kTile = kPanels * kPanelBytes;   // 128 x D bf16
+    static constexpr uint32_t kHalfDS = 128 * 128;             // [128 kv][64 q] bf16
     static constexpr uint32_t kK = 0;
     static constexpr uint32_t kV = kK + kTile;
-    static constexpr uint32_t kQ = kV + kTile;
-    static constexpr uint32_t kDO = kQ + kTile;
-    static constexpr uint32_t kPt = kDO + kTile;               // 128 x 128 bf16
-    static constexpr uint32_t kDSt = kPt + 2 * kPanelBytes;    // 128 x 128 bf16
-    static constexpr uint32_t kVec = kDSt + 2 * kPanelBytes;   // lse2, D, w: 3 x 128 fp32
-    static constexpr uint32_t kBars = kVec + 3 * 128 * 4;
-    static constexpr uint32_t kBytes = kBars + 64;
+    static constexpr uint32_t kQdo = kV + kTile;               // stage s: Q at +2s*kTile, dO at +(2s+1)*kTile
+    static constexpr uint32_t kDS = kQdo + 4 * kTile;          // two halves
+    static constexpr uint32_t kVec = kDS + 2 * kHalfDS;        // lse*log2e [128], D [128]
+    static constexpr uint32_t kBars = kVec + 2 * 128 * 4;
+    static constexpr uint32_t kBytes = kBars + 256;
     static constexpr uint32_t kAlloc = kBytes + 1024;
 };
 
-constexpr int kBwdThreads = 128;
+constexpr int kBwdThreads = 384;
+
+// One (query head, query tile) pair of a KV tile's walk, published by the
+// producer warp so that no other role reads the kept lists from global memory.
+// h < 0 marks the end of the walk.
+struct PairEntry {
+    int h, tile;
+    float w0, w1;   // block weights of the tile's two 64-row halves
+};
 
 // Walks the kept query tiles of one (segment, KV head) group in ascending order
-// of (head in group, tile).  Every thread runs the same walk.
+// of (head in group, tile).  Every role runs its own copy of the same walk.
 struct KeptTileWalk {
     const int32_t* kept_idx;
     const int32_t* kept_cnt;
@@ -67,6 +82,18 @@ struct KeptTileWalk {
     const int32_t* list;
     int tile, h;
 
+    __device__ void init(const BwdParams& p, int G_, int g_, int s_, int jt, int len) {
+        kept_idx = p.kept_idx;
+        kept_cnt = p.kept_cnt;
+        nbmax = p.nbmax;
+        hq = p.hq;
+        G = G_;
+        g = g_;
+        s = s_;
+        block_q = p.block_q;
+        first_block = p.causal ? (jt * 128) / p.block_q : 0;
+        nb = (len + p.block_q - 1) / p.block_q;
+    }
     __device__ void open_head() {
         h = g * G + hh;
         const size_t base = ((size_t)s * hq + h) * nbmax;
@@ -104,6 +131,13 @@ struct KeptTileWalk {
     }
 };
 
+// Weight of the query rows [q0, q0 + 64) of a tile (one selection block, or
+// half of one): 0 past the segment's end.
+__device__ __forceinline__ float half_weight(const BwdParams& p, int s, int h, int q0, int len) {
+    if (q0 >= len) return 0.f;
+    return p.block_weight[((size_t)s * p.hq + h) * p.nbmax + q0 / p.block_q];
+}
+
 template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -114,28 +148,45 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* lse2_s = reinterpret_cast<float*>(smem + L::kVec);
     float* dvec_s = lse2_s + 128;
-    float* w_s = dvec_s + 128;
-    uint64_t* bar_kv = reinterpret_cast<uint64_t*>(smem + L::kBars);
-    uint64_t* bar_qdo = bar_kv + 1;
-    uint64_t* bar_mma = bar_kv + 2;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_kv + 3);
-    int* abort_flag = reinterpret_cast<int*>(bar_kv + 4);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
+    uint64_t* bar_kv = bars + 0;
+    uint64_t* bar_qdo_full = bars + 1;    // [2] stages
+    uint64_t* bar_qdo_empty = bars + 3;   // [2]
+    uint64_t* bar_s_full = bars + 5;      // [2] halves
+    uint64_t* bar_p_ready = bars + 7;     // [2]
+    uint64_t* bar_dq_full = bars + 9;     // [2]
+    uint64_t* bar_dq_free = bars + 11;    // [2]
+    uint64_t* bar_done = bars + 13;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 14);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 15);
+    uint64_t* bar_entry = bars + 16;      // [4] work-list ring
+    PairEntry* ring = reinterpret_cast<PairEntry*>(bars + 20);   // [4] x 16 B
 
-    const int g = blockIdx.x;
-    const int jt = blockIdx.y;              // KV tile: lowest index = most work, first
+    // KV tile fastest: CTAs resident together share one KV head's group, so its
+    // Q/dO stay in L2; within a group the lowest tiles (most work) start first
+    const int jt = blockIdx.x;
+    const int g = blockIdx.y;
     const int s = blockIdx.z;
     int seg0, len;
     if (!load_segment(prm.cu_seqlens, s, prm.T, prm.max_seqlen, seg0, len, 30)) return;
     if (jt * 128 >= len) return;
     const int G = prm.hq / prm.hkv;
 
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t s_base = smem_addr(smem);
 
     if (tid == 0) {
         mbar_init(bar_kv, 1);
-        mbar_init(bar_qdo, 1);
-        mbar_init(bar_mma, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bar_qdo_full[i], 1);
+            mbar_init(&bar_qdo_empty[i], 1);
+            mbar_init(&bar_s_full[i], 1);
+            mbar_init(&bar_p_ready[i], 128);
+            mbar_init(&bar_dq_full[i], 1);
+            mbar_init(&bar_dq_free[i], 128);
+        }
+        mbar_init(bar_done, 1);
+        for (int i = 0; i < 4; ++i) mbar_init(&bar_entry[i], 1);
         *abort_flag = 0;
         fence_barrier_init();
         prefetch_tensormap(&tm_q);
@@ -151,203 +202,248 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t t_st = tmem;               // S^T   [0, 128)
-    const uint32_t t_dpt = tmem + 128;        // dP^T  [128, 256)
-    const uint32_t t_dv = tmem + 256;         // dV    [256, 256 + D)
-    const uint32_t t_dk = tmem + 256 + D;     // dK    [256 + D, 256 + 2D)
-    const uint32_t t_dq = tmem;               // partial dQ reuses S^T's columns
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
-
+    const uint32_t t_dv = tmem;
+    const uint32_t t_dk = tmem + 128;
     const int kv_row0 = seg0 + jt * 128;
 
+    // Does this KV tile have any work?  (every role sees the same answer)
     KeptTileWalk walk;
-    walk.kept_idx = prm.kept_idx;
-    walk.kept_cnt = prm.kept_cnt;
-    walk.nbmax = prm.nbmax;
-    walk.hq = prm.hq;
-    walk.G = G;
-    walk.g = g;
-    walk.s = s;
-    walk.block_q = prm.block_q;
-    walk.first_block = prm.causal ? (jt * 128) / prm.block_q : 0;
-    walk.nb = (len + prm.block_q - 1) / prm.block_q;
+    walk.init(prm, G, g, s, jt, len);
+    const bool any = walk.next(true);
 
-    constexpr uint32_t kIdescT = idesc_bf16(128, 128, 0, 0);   // S^T, dP^T
-    constexpr uint32_t kIdescKV = idesc_bf16(128, D, 0, 1);     // dV, dK: B (dO, Q) MN-major
-    constexpr uint32_t kIdescQ = idesc_bf16(128, D, 1, 1);      // dQ: A (dS) and B (K) MN-major
-    const int kv_local = jt * 128 + tid;    // this thread's KV row (S^T/dP^T/dV/dK lane)
-    const bool kv_valid = kv_local < len;
+    constexpr uint32_t kIdescS = idesc_bf16(128, 64, 0, 0);    // S^T, dP^T halves
+    constexpr uint32_t kIdescKV = idesc_bf16(128, D, 0, 1);    // dV, dK (A from TMEM, B MN-major)
+    constexpr uint32_t kIdescQ = idesc_bf16(128, 64, 1, 1);    // dQ^T half (A K^T, B dS^T: MN-major)
 
-    uint32_t ph_qdo = 0, ph_mma = 0;
-    bool kv_waited = false, ok = true;
-    int n_iter = 0;
-    int qdo_pending = 0;   // thread 0: Q/dO loads issued but not yet waited on
-
-    bool more = walk.next(true);
-    if (more && tid == 0) {
-        mbar_arrive_expect_tx(bar_kv, 2 * L::kTile);
-        for (int c = 0; c < L::kPanels; ++c) {
-            tma_load_3d(smem + L::kK + c * kPanelBytes, &tm_k, bar_kv, c * 64, g, kv_row0);
-            tma_load_3d(smem + L::kV + c * kPanelBytes, &tm_v, bar_kv, c * 64, g, kv_row0);
-        }
-        mbar_arrive_expect_tx(bar_qdo, 2 * L::kTile);
-        ++qdo_pending;
-        for (int c = 0; c < L::kPanels; ++c) {
-            tma_load_3d(smem + L::kQ + c * kPanelBytes, &tm_q, bar_qdo, c * 64, walk.h, seg0 + walk.tile * 128);
-            tma_load_3d(smem + L::kDO + c * kPanelBytes, &tm_do, bar_qdo, c * 64, walk.h, seg0 + walk.tile * 128);
-        }
-    }
-
-    while (more) {
-        const int h = walk.h, qt = walk.tile;
-        // per-column (query row) vectors of this tile
-        {
-            const int q_local = qt * 128 + tid;
-            float l2 = 0.f, dd = 0.f, w = 0.f;
-            if (q_local < len) {
-                const size_t idx = (size_t)h * prm.T + seg0 + q_local;
-                l2 = prm.lse[idx] * 1.4426950408889634f;
-                dd = prm.Dvec[idx];
-                w = prm.block_weight[((size_t)s * prm.hq + h) * prm.nbmax + q_local / prm.block_q];
+    if (warp == 0) {
+        // ===================== TMA producer + work list =====================
+        if (lane == 0) {
+            uint32_t fill_parity[2] = {0, 0};
+            bool filled[2] = {false, false};
+            if (any) {
+                mbar_arrive_expect_tx(bar_kv, 2 * L::kTile);
+                for (int c = 0; c < L::kPanels; ++c) {
+                    tma_load_3d(smem + L::kK + c * kPanelBytes, &tm_k, bar_kv, c * 64, g, kv_row0);
+                    tma_load_3d(smem + L::kV + c * kPanelBytes, &tm_v, bar_kv, c * 64, g, kv_row0);
+                }
             }
-            lse2_s[tid] = l2;
-            dvec_s[tid] = dd;
-            w_s[tid] = w;
-        }
-        if (tid == 0) {
-            bool w_ok = kv_waited || mbar_wait(bar_kv, 0, 11);
-            kv_waited = w_ok;
-            w_ok = w_ok && mbar_wait(bar_qdo, ph_qdo, 12);
-            if (w_ok) {
-                --qdo_pending;
-                ph_qdo ^= 1;
-                tc_fence_after();
-                const uint32_t ka = s_base + L::kK, va = s_base + L::kV;
-                const uint32_t qa = s_base + L::kQ, da = s_base + L::kDO;
-#pragma unroll
-                for (int k = 0; k < D / 16; ++k)
-                    mma_bf16_ss(t_st, desc_kmajor(ka, k), desc_kmajor(qa, k), kIdescT, k > 0);
-#pragma unroll
-                for (int k = 0; k < D / 16; ++k)
-                    mma_bf16_ss(t_dpt, desc_kmajor(va, k), desc_kmajor(da, k), kIdescT, k > 0);
-                mma_commit(bar_mma);
-            } else {
-                *abort_flag = 1;
+            int n = 0;
+            bool more = any, ok = true;
+            while (more) {
+                const int st = n & 1;
+                // the stage (and, by the pipeline's order, ring slot n % 4) is free
+                if (n >= 2 && !mbar_wait_or_abort(&bar_qdo_empty[st], ((n >> 1) - 1) & 1, 31, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                const int q0 = walk.tile * 128;
+                PairEntry e;
+                e.h = walk.h;
+                e.tile = walk.tile;
+                e.w0 = half_weight(prm, s, walk.h, q0, len);
+                e.w1 = half_weight(prm, s, walk.h, q0 + 64, len);
+                ring[n & 3] = e;
+                mbar_arrive(&bar_entry[n & 3]);
+                const int row = seg0 + q0;
+                mbar_arrive_expect_tx(&bar_qdo_full[st], 2 * L::kTile);
+                for (int c = 0; c < L::kPanels; ++c) {
+                    tma_load_3d(smem + L::kQdo + (2 * st) * L::kTile + c * kPanelBytes, &tm_q,
+                                &bar_qdo_full[st], c * 64, walk.h, row);
+                    tma_load_3d(smem + L::kQdo + (2 * st + 1) * L::kTile + c * kPanelBytes, &tm_do,
+                                &bar_qdo_full[st], c * 64, walk.h, row);
+                }
+                fill_parity[st] = (n >> 1) & 1;
+                filled[st] = true;
+                ++n;
+                more = walk.next(false);
+            }
+            // end-of-walk entry (slot n % 4 was last used by pair n - 4)
+            if (ok && n >= 2 &&
+                !mbar_wait_or_abort(&bar_qdo_empty[n & 1], ((n >> 1) - 1) & 1, 31, abort_flag))
+                ok = false;
+            if (ok) {
+                PairEntry e;
+                e.h = -1;
+                e.tile = 0;
+                e.w0 = e.w1 = 0.f;
+                ring[n & 3] = e;
+                mbar_arrive(&bar_entry[n & 3]);
+            }
+            if (*abort_flag) {
+                // let this CTA's own copies land before the CTA exits (bounded)
+                if (any) mbar_wait(bar_kv, 0, 32);
+                for (int st = 0; st < 2; ++st)
+                    if (filled[st]) mbar_wait(&bar_qdo_full[st], fill_parity[st], 32);
             }
         }
-        __syncthreads();
-        if (*abort_flag) { ok = false; break; }
-        if (!mbar_wait(bar_mma, ph_mma, 13)) *abort_flag = 1;
-        ph_mma ^= 1;
-        __syncthreads();
-        if (*abort_flag) { ok = false; break; }
-        tc_fence_after();
-
-        // ---- P^T and dS^T for this thread's KV row ----
-        const uint32_t pt_base = s_base + L::kPt, dst_base = s_base + L::kDSt;
-        const int q0 = qt * 128;
-#pragma unroll 1
-        for (int c = 0; c < 4; ++c) {
-            float sv[32], dpv[32];
-            tmem_ld32(t_st + lane_off + c * 32, sv);
-            tmem_ld32(t_dpt + lane_off + c * 32, dpv);
-#pragma unroll
-            for (int ch = 0; ch < 4; ++ch) {
-                uint32_t pk[4], dk_[4];
-#pragma unroll
-                for (int e2 = 0; e2 < 4; ++e2) {
-                    float pv[2], dsv[2];
-#pragma unroll
-                    for (int u = 0; u < 2; ++u) {
-                        const int col = c * 32 + ch * 8 + e2 * 2 + u;
-                        const int q_local = q0 + col;
-                        const bool valid = kv_valid && q_local < len && (!prm.causal || kv_local <= q_local);
-                        const float p = valid ? fast_exp2(sv[ch * 8 + e2 * 2 + u] * prm.scale_log2 - lse2_s[col]) : 0.f;
-                        const float w = w_s[col];
-                        pv[u] = p * w;
-                        dsv[u] = p * (dpv[ch * 8 + e2 * 2 + u] - dvec_s[col]) * w;
+        __syncwarp();
+    } else if (warp == 1) {
+        // ===================== MMA issuer (one thread) =====================
+        if (lane == 0 && any) {
+            const uint32_t ka = s_base + L::kK, va = s_base + L::kV;
+            const bool ok = mbar_wait_or_abort(bar_kv, 0, 33, abort_flag);
+            int n = 0;
+            bool more = ok;
+            while (more) {
+                const int st = n & 1;
+                if (!mbar_wait_or_abort(&bar_entry[n & 3], (n >> 2) & 1, 34, abort_flag)) break;
+                if (ring[n & 3].h < 0) break;
+                if (!mbar_wait_or_abort(&bar_qdo_full[st], (n >> 1) & 1, 34, abort_flag)) break;
+                const uint32_t qa = s_base + L::kQdo + (2 * st) * L::kTile;
+                const uint32_t da = qa + L::kTile;
+                // S^T and dP^T of both halves
+                bool w_ok = true;
+                for (int hf = 0; hf < 2; ++hf) {
+                    if (n > 0 && !mbar_wait_or_abort(&bar_dq_free[hf], (n - 1) & 1, 35, abort_flag)) {
+                        w_ok = false;
+                        break;
                     }
-                    pk[e2] = pack_bf16(pv[0], pv[1]);
-                    dk_[e2] = pack_bf16(dsv[0], dsv[1]);
+                    tc_fence_after();
+                    const uint32_t t_s = tmem + 256 + hf * 128, t_dp = t_s + 64;
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k)
+                        mma_bf16_ss(t_s, desc_kmajor(ka, k), desc_kmajor(qa + hf * 8192, k), kIdescS, k > 0);
+#pragma unroll
+                    for (int k = 0; k < D / 16; ++k)
+                        mma_bf16_ss(t_dp, desc_kmajor(va, k), desc_kmajor(da + hf * 8192, k), kIdescS, k > 0);
+                    mma_commit(&bar_s_full[hf]);
                 }
-                const uint32_t off = sw128_chunk_offset(tid, c * 4 + ch);
-                st_shared_v4(pt_base + off, pk[0], pk[1], pk[2], pk[3]);
-                st_shared_v4(dst_base + off, dk_[0], dk_[1], dk_[2], dk_[3]);
-            }
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t ka = s_base + L::kK;
-            const uint32_t qa = s_base + L::kQ, da = s_base + L::kDO;
+                if (!w_ok) break;
+                // dV, dK (TS) and dQ^T (SS) of both halves
+                for (int hf = 0; hf < 2; ++hf) {
+                    if (!mbar_wait_or_abort(&bar_p_ready[hf], n & 1, 36, abort_flag)) {
+                        w_ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t t_s = tmem + 256 + hf * 128, t_dp = t_s + 64;
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-                mma_bf16_ss(t_dv, desc_kmajor(pt_base, k), desc_mnmajor(da, k), kIdescKV,
-                            (n_iter > 0 || k > 0) ? 1u : 0u);
+                    for (int k = 0; k < 4; ++k)
+                        mma_bf16_ts(t_dv, t_s + k * 8, desc_mnmajor(da, hf * 4 + k), kIdescKV,
+                                    (n > 0 || hf > 0 || k > 0) ? 1u : 0u);
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-                mma_bf16_ss(t_dk, desc_kmajor(dst_base, k), desc_mnmajor(qa, k), kIdescKV,
-                            (n_iter > 0 || k > 0) ? 1u : 0u);
+                    for (int k = 0; k < 4; ++k)
+                        mma_bf16_ts(t_dk, t_dp + k * 8, desc_mnmajor(qa, hf * 4 + k), kIdescKV,
+                                    (n > 0 || hf > 0 || k > 0) ? 1u : 0u);
+                    if (hf == 1) mma_commit(&bar_qdo_empty[st]);   // Q/dO of this stage fully read
+                    const uint32_t dsa = s_base + L::kDS + hf * L::kHalfDS;
 #pragma unroll
-            for (int k = 0; k < 8; ++k)
-                mma_bf16_ss(t_dq, desc_mnmajor(dst_base, k), desc_mnmajor(ka, k), kIdescQ, k > 0);
-            mma_commit(bar_mma);
-        }
-        if (!mbar_wait(bar_mma, ph_mma, 14)) *abort_flag = 1;
-        ph_mma ^= 1;
-        // the walk's next tile: its Q/dO load overlaps the dQ reduction below
-        more = walk.next(false);
-        __syncthreads();
-        if (*abort_flag) { ok = false; break; }
-        tc_fence_after();
-        if (more && tid == 0) {
-            mbar_arrive_expect_tx(bar_qdo, 2 * L::kTile);
-            ++qdo_pending;
-            for (int c = 0; c < L::kPanels; ++c) {
-                tma_load_3d(smem + L::kQ + c * kPanelBytes, &tm_q, bar_qdo, c * 64, walk.h, seg0 + walk.tile * 128);
-                tma_load_3d(smem + L::kDO + c * kPanelBytes, &tm_do, bar_qdo, c * 64, walk.h, seg0 + walk.tile * 128);
-            }
-        }
-
-        // ---- partial dQ of this tile: thread r owns query row r ----
-        {
-            const int q_local = q0 + tid;
-            const bool row_ok = q_local < len && w_s[tid] != 0.f;
-            float* dst = prm.dq_acc + ((size_t)(seg0 + q_local) * prm.hq + h) * D;
-#pragma unroll 1
-            for (int c = 0; c < D / 32; ++c) {
-                float v[32];
-                tmem_ld32(t_dq + lane_off + c * 32, v);
-                if (row_ok) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        atomicAdd(reinterpret_cast<float4*>(dst + c * 32 + e * 4),
-                                  make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]));
+                    for (int k = 0; k < 8; ++k) {
+                        // A = K^T (M = d): MN-major over the K tile; with d = 64 the
+                        // second 64-row atom repeats the first (those lanes are unused)
+                        const uint64_t adesc =
+                            (D == 128) ? desc_mnmajor(ka, k) : sw128_desc(ka + k * 2048, 0, 1024);
+                        mma_bf16_ss(t_s, adesc, desc_mnmajor(dsa, k), kIdescQ, k > 0);
+                    }
+                    mma_commit(&bar_dq_full[hf]);
                 }
+                if (!w_ok) break;
+                ++n;
             }
+            mma_commit(bar_done);
+            // every MMA this thread issued must finish before TMEM is released
+            mbar_wait(bar_done, 0, 37);
         }
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        ++n_iter;
-    }
-
-    if (ok) {
+        __syncwarp();
+    } else if (warp >= 4 && warp < 8) {
+        // ===================== element-wise (thread = KV row) =====================
+        const int r = tid - 128;                          // TMEM lane / KV row
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const int kv_local = jt * 128 + r;
+        const bool kv_valid = kv_local < len;
+        int n = 0;
+        bool more = any, failed = false;
+        for (;;) {
+            // uniform decision of the four warps; also: all are done with the old vectors
+            if (named_bar_or(1, 128, !more || failed)) break;
+            const bool got_e = mbar_wait_or_abort(&bar_entry[n & 3], (n >> 2) & 1, 41, abort_flag);
+            const PairEntry e = ring[n & 3];
+            if (!got_e || e.h < 0) {
+                more = false;
+                failed = !got_e;
+                continue;
+            }
+            const int h = e.h, qt = e.tile, q0 = qt * 128;
+            {
+                const int q_local = q0 + r;
+                float l2 = INFINITY, dd = 0.f;    // exp2(S - inf) = 0: columns past the segment vanish
+                if (q_local < len) {
+                    const size_t idx = (size_t)h * prm.T + seg0 + q_local;
+                    l2 = prm.lse[idx] * 1.4426950408889634f;
+                    dd = prm.Dvec[idx];
+                }
+                lse2_s[r] = l2;
+                dvec_s[r] = dd;
+            }
+            named_bar_sync(1, 128);
+            const bool diag = prm.causal && qt == jt;
+            for (int hf = 0; hf < 2 && !failed; ++hf) {
+                const float w = kv_valid ? (hf ? e.w1 : e.w0) : 0.f;
+                const bool got = mbar_wait_or_abort(&bar_s_full[hf], n & 1, 38, abort_flag);
+                if (!__all_sync(0xffffffffu, got)) { failed = true; break; }
+                tc_fence_after();
+                const uint32_t t_s = tmem + 256 + hf * 128 + lane_off, t_dp = t_s + 64;
+                const uint32_t dsa = s_base + L::kDS + hf * L::kHalfDS;
+#pragma unroll
+                for (int c = 0; c < 2; ++c) {
+                    float sv[32], dpv[32];
+                    tmem_ld32(t_s + c * 32, sv);
+                    tmem_ld32(t_dp + c * 32, dpv);
+                    uint32_t pk[16], dk_[16];
+#pragma unroll
+                    for (int e4 = 0; e4 < 8; ++e4) {
+                        const int col0 = hf * 64 + c * 32 + 4 * e4;
+                        const float4 l4 = *reinterpret_cast<const float4*>(lse2_s + col0);
+                        const float4 d4 = *reinterpret_cast<const float4*>(dvec_s + col0);
+                        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                        const float dv_[4] = {d4.x, d4.y, d4.z, d4.w};
+                        float pw[4], dsw[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            float p = fast_exp2(fmaf(sv[4 * e4 + u], prm.scale_log2, -lv[u]));
+                            if (diag && kv_local > q0 + col0 + u) p = 0.f;
+                            pw[u] = p * w;
+                            dsw[u] = pw[u] * (dpv[4 * e4 + u] - dv_[u]);
+                        }
+                        pk[2 * e4] = pack_bf16(pw[0], pw[1]);
+                        pk[2 * e4 + 1] = pack_bf16(pw[2], pw[3]);
+                        dk_[2 * e4] = pack_bf16(dsw[0], dsw[1]);
+                        dk_[2 * e4 + 1] = pack_bf16(dsw[2], dsw[3]);
+                    }
+                    // P^T over S^T (packed columns [16c, 16c+16)), dS^T over dP^T
+                    tmem_st16(t_s + c * 16, pk);
+                    tmem_st16(t_dp + c * 16, dk_);
+                    // dS^T into shared memory (one 64-column panel, SW128)
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch)
+                        st_shared_v4(dsa + sw128_chunk_offset(r, c * 4 + ch), dk_[4 * ch],
+                                     dk_[4 * ch + 1], dk_[4 * ch + 2], dk_[4 * ch + 3]);
+                }
+                tmem_wait_st();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&bar_p_ready[hf]);
+            }
+            if (!failed) ++n;
+        }
         // ---- epilogue: dV, dK (x softmax_scale) for this thread's KV row ----
-        const size_t orow = ((size_t)(kv_row0 + tid) * prm.hkv + g) * D;
+        bool have = n > 0 && !failed && !*abort_flag;
+        if (have) have = mbar_wait_or_abort(bar_done, 0, 39, abort_flag);
+        have = __all_sync(0xffffffffu, have);
+        tc_fence_after();
+        const bool write = kv_valid && (have || (n == 0 && !failed));
+        const size_t orow = ((size_t)(kv_row0 + r) * prm.hkv + g) * D;
 #pragma unroll 1
         for (int c = 0; c < D / 32; ++c) {
             float v[32], k[32];
-            if (n_iter > 0) {
+            if (have) {
                 tmem_ld32(t_dv + lane_off + c * 32, v);
                 tmem_ld32(t_dk + lane_off + c * 32, k);
             } else {
 #pragma unroll
                 for (int e = 0; e < 32; ++e) { v[e] = 0.f; k[e] = 0.f; }
             }
-            if (kv_valid) {
+            if (write) {
 #pragma unroll
                 for (int e8 = 0; e8 < 4; ++e8) {
                     uint4 pv, pk;
@@ -364,14 +460,54 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 }
             }
         }
-    } else if (tid == 0) {
-        // a wait gave up: let this CTA's own TMA copies land (bounded) before exit
-        if (!kv_waited && n_iter == 0) mbar_wait(bar_kv, 0, 15);
-        while (qdo_pending > 0 && mbar_wait(bar_qdo, ph_qdo, 15)) { --qdo_pending; ph_qdo ^= 1; }
+    } else if (warp >= 8) {
+        // ===================== dQ drain (thread = head-dim index) =====================
+        const int dd = tid - 256;                         // TMEM lane = d index
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const bool lane_used = (warp & 3) * 32 < D;       // d = 64: warps 10, 11 idle
+        const size_t row_stride = (size_t)prm.hq * D;
+        int n = 0;
+        bool more = any;
+        while (more) {
+            const bool got_e = mbar_wait_or_abort(&bar_entry[n & 3], (n >> 2) & 1, 42, abort_flag);
+            if (!__all_sync(0xffffffffu, got_e)) break;
+            const PairEntry e = ring[n & 3];
+            if (e.h < 0) break;
+            const int h = e.h, q0 = e.tile * 128;
+            bool ok = true;
+            for (int hf = 0; hf < 2; ++hf) {
+                const bool got = mbar_wait_or_abort(&bar_dq_full[hf], n & 1, 40, abort_flag);
+                if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                tc_fence_after();
+                const int qh = q0 + hf * 64;
+                const bool live = lane_used && qh < len && (hf ? e.w1 : e.w0) != 0.f;
+                if (live) {
+                    const uint32_t t_q = tmem + 256 + hf * 128 + lane_off;
+                    float* dst = prm.dq_acc + ((size_t)(seg0 + qh) * prm.hq + h) * D + dd;
+                    const int nvalid = min(64, len - qh);
+#pragma unroll
+                    for (int c = 0; c < 2; ++c) {
+                        float v[32];
+                        tmem_ld32(t_q + c * 32, v);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            if (c * 32 + e < nvalid) atomicAdd(dst + (size_t)(c * 32 + e) * row_stride, v[e]);
+                    }
+                }
+                tc_fence_before();
+                mbar_arrive(&bar_dq_free[hf]);
+            }
+            if (!ok) break;
+            ++n;
+        }
     }
+
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 512);
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
 }
 
 }  // namespace lf
