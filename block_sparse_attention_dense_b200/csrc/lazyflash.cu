@@ -132,6 +132,21 @@ lf_status launch_bwd(const lf_attn_desc* d, const void* q, const void* k, const 
         !make_thd_map(&mv, v, d->total_tokens, d->hkv, D) ||
         !make_thd_map(&mdo, dout, d->total_tokens, d->hq, D))
         return LF_ERR_CUDA;
+    // fp32 accumulator [T][hq][D] as a 3-D map (D, hq, T) with 32-row boxes: the
+    // backward adds staged dQ tiles into it by TMA reduction
+    CUtensorMap mdq;
+    {
+        EncodeTiledFn enc = encode_tiled();
+        if (!enc) return LF_ERR_CUDA;
+        const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)d->hq, (cuuint64_t)d->total_tokens};
+        const cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)d->hq * D * 4};
+        const cuuint32_t box[3] = {(cuuint32_t)D, 1, 32};
+        const cuuint32_t estr[3] = {1, 1, 1};
+        if (enc(&mdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, dq_acc, dims, strides, box, estr,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return LF_ERR_CUDA;
+    }
     const size_t nacc = (size_t)d->total_tokens * d->hq * D;
     if (cudaMemsetAsync(dq_acc, 0, nacc * sizeof(float), st) != cudaSuccess) return LF_ERR_CUDA;
     lf::BwdParams p{};
@@ -158,7 +173,7 @@ lf_status launch_bwd(const lf_attn_desc* d, const void* q, const void* k, const 
                              smem) != cudaSuccess)
         return LF_ERR_CUDA;
     dim3 grid(ntiles_of(d), d->hkv, d->nseq);
-    lf::attn_bwd_kernel<D><<<grid, lf::kBwdThreads, smem, st>>>(mq, mk, mv, mdo, p);
+    lf::attn_bwd_kernel<D><<<grid, lf::kBwdThreads, smem, st>>>(mq, mk, mv, mdo, mdq, p);
     if (launch_status() != LF_OK) return LF_ERR_CUDA;
     const size_t n8 = nacc / 8;
     const int blocks = (int)std::min<size_t>((n8 + 255) / 256, 148 * 16);

@@ -142,7 +142,7 @@ template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    BwdParams prm) {
+                    const __grid_constant__ CUtensorMap tm_dq, BwdParams prm) {
     using L = BwdSmem<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -193,6 +193,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
         prefetch_tensormap(&tm_do);
+        prefetch_tensormap(&tm_dq);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, 512);
@@ -384,15 +385,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tc_fence_after();
                 const uint32_t t_s = tmem + 256 + hf * 128 + lane_off, t_dp = t_s + 64;
                 const uint32_t dsa = s_base + L::kDS + hf * L::kHalfDS;
+                // 16-column chunks; the next chunk's TMEM loads overlap this chunk's math
+                auto chunk = [&](int c, const uint32_t (&sr)[16], const uint32_t (&dr)[16]) {
+                    uint32_t pk[8], dk_[8];
 #pragma unroll
-                for (int c = 0; c < 2; ++c) {
-                    float sv[32], dpv[32];
-                    tmem_ld32(t_s + c * 32, sv);
-                    tmem_ld32(t_dp + c * 32, dpv);
-                    uint32_t pk[16], dk_[16];
-#pragma unroll
-                    for (int e4 = 0; e4 < 8; ++e4) {
-                        const int col0 = hf * 64 + c * 32 + 4 * e4;
+                    for (int e4 = 0; e4 < 4; ++e4) {
+                        const int col0 = hf * 64 + c * 16 + 4 * e4;
                         const float4 l4 = *reinterpret_cast<const float4*>(lse2_s + col0);
                         const float4 d4 = *reinterpret_cast<const float4*>(dvec_s + col0);
                         const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
@@ -400,25 +398,41 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         float pw[4], dsw[4];
 #pragma unroll
                         for (int u = 0; u < 4; ++u) {
-                            float p = fast_exp2(fmaf(sv[4 * e4 + u], prm.scale_log2, -lv[u]));
+                            float p = fast_exp2(fmaf(__uint_as_float(sr[4 * e4 + u]), prm.scale_log2, -lv[u]));
                             if (diag && kv_local > q0 + col0 + u) p = 0.f;
                             pw[u] = p * w;
-                            dsw[u] = pw[u] * (dpv[4 * e4 + u] - dv_[u]);
+                            dsw[u] = pw[u] * (__uint_as_float(dr[4 * e4 + u]) - dv_[u]);
                         }
                         pk[2 * e4] = pack_bf16(pw[0], pw[1]);
                         pk[2 * e4 + 1] = pack_bf16(pw[2], pw[3]);
                         dk_[2 * e4] = pack_bf16(dsw[0], dsw[1]);
                         dk_[2 * e4 + 1] = pack_bf16(dsw[2], dsw[3]);
                     }
-                    // P^T over S^T (packed columns [16c, 16c+16)), dS^T over dP^T
-                    tmem_st16(t_s + c * 16, pk);
-                    tmem_st16(t_dp + c * 16, dk_);
+                    // P^T over S^T (packed columns [8c, 8c+8)), dS^T over dP^T: columns
+                    // whose fp32 values were read by earlier chunks
+                    tmem_st8(t_s + c * 8, pk);
+                    tmem_st8(t_dp + c * 8, dk_);
                     // dS^T into shared memory (one 64-column panel, SW128)
-#pragma unroll
-                    for (int ch = 0; ch < 4; ++ch)
-                        st_shared_v4(dsa + sw128_chunk_offset(r, c * 4 + ch), dk_[4 * ch],
-                                     dk_[4 * ch + 1], dk_[4 * ch + 2], dk_[4 * ch + 3]);
-                }
+                    st_shared_v4(dsa + sw128_chunk_offset(r, 2 * c), dk_[0], dk_[1], dk_[2], dk_[3]);
+                    st_shared_v4(dsa + sw128_chunk_offset(r, 2 * c + 1), dk_[4], dk_[5], dk_[6], dk_[7]);
+                };
+                uint32_t sa[16], da[16], sb[16], db[16];
+                tmem_ld16_nowait(t_s, sa);
+                tmem_ld16_nowait(t_dp, da);
+                tmem_wait_ld_regs(sa, da);
+                tmem_ld16_nowait(t_s + 16, sb);
+                tmem_ld16_nowait(t_dp + 16, db);
+                chunk(0, sa, da);
+                tmem_wait_ld_regs(sb, db);
+                tmem_ld16_nowait(t_s + 32, sa);
+                tmem_ld16_nowait(t_dp + 32, da);
+                chunk(1, sb, db);
+                tmem_wait_ld_regs(sa, da);
+                tmem_ld16_nowait(t_s + 48, sb);
+                tmem_ld16_nowait(t_dp + 48, db);
+                chunk(2, sa, da);
+                tmem_wait_ld_regs(sb, db);
+                chunk(3, sb, db);
                 tmem_wait_st();
                 fence_proxy_async_smem();
                 tc_fence_before();
@@ -465,7 +479,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const int dd = tid - 256;                         // TMEM lane = d index
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const bool lane_used = (warp & 3) * 32 < D;       // d = 64: warps 10, 11 idle
-        const size_t row_stride = (size_t)prm.hq * D;
         int n = 0;
         bool more = any;
         while (more) {
@@ -480,18 +493,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
                 tc_fence_after();
                 const int qh = q0 + hf * 64;
-                const bool live = lane_used && qh < len && (hf ? e.w1 : e.w0) != 0.f;
+                const bool live = qh < len && (hf ? e.w1 : e.w0) != 0.f;
                 if (live) {
+                    // The half's dS^T buffer is idle from the end of its dQ^T MMA until
+                    // dq_free: stage 32 query rows x d fp32 there and let TMA add them
+                    // into the accumulator (rows past T are clipped by TMA; rows past
+                    // the segment carry exact zeros).
+                    float* stage = reinterpret_cast<float*>(smem + L::kDS + hf * L::kHalfDS);
                     const uint32_t t_q = tmem + 256 + hf * 128 + lane_off;
-                    float* dst = prm.dq_acc + ((size_t)(seg0 + qh) * prm.hq + h) * D + dd;
-                    const int nvalid = min(64, len - qh);
+                    for (int rnd = 0; rnd < 2; ++rnd) {
+                        if (qh + rnd * 32 >= len) break;
+                        if (lane_used) {
+                            float v[32];
+                            tmem_ld32(t_q + rnd * 32, v);
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        float v[32];
-                        tmem_ld32(t_q + c * 32, v);
-#pragma unroll
-                        for (int e = 0; e < 32; ++e)
-                            if (c * 32 + e < nvalid) atomicAdd(dst + (size_t)(c * 32 + e) * row_stride, v[e]);
+                            for (int q = 0; q < 32; ++q) stage[q * D + dd] = v[q];
+                        }
+                        fence_proxy_async_smem();
+                        named_bar_sync(2, 128);
+                        if (dd == 0) {
+                            tma_reduce_add_3d(&tm_dq, stage, 0, h, seg0 + qh + rnd * 32);
+                            bulk_commit_group();
+                            bulk_wait_read0();
+                        }
+                        named_bar_sync(2, 128);   // the stage may be written again
                     }
                 }
                 tc_fence_before();
@@ -500,6 +525,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!ok) break;
             ++n;
         }
+        if (dd == 0) bulk_wait0();   // reductions performed before the CTA retires
     }
 
     tc_fence_before();
