@@ -350,7 +350,7 @@ def main():
                      "traffic": traffic.get(dom.split()[0])},
         "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / Ke, "steps": Ke},
-        "gpu_launches": 5 * K,
+        "gpu_launches": 7 * K,   # fwd, norms, select, bwd, 3 accumulator conversions
         "clocks": clk,
     }
     if rank == 0 and n == 1 and not args.no_cpu_baseline:

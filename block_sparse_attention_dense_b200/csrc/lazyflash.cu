@@ -58,12 +58,25 @@ lf_status check_desc(const lf_attn_desc* d) {
 inline int nbmax_of(const lf_attn_desc* d) { return (d->max_seqlen + d->block_q - 1) / d->block_q; }
 inline int ntiles_of(const lf_attn_desc* d) { return (d->max_seqlen + 127) / 128; }
 
-size_t bwd_ws_bytes(const lf_attn_desc* d, bool need_D) {
-    size_t b = (size_t)d->total_tokens * d->hq * d->d * sizeof(float);   // fp32 dQ accumulator
-    b = (b + 255) & ~size_t(255);
-    if (need_D) b += ((size_t)d->total_tokens * d->hq * sizeof(float) + 255) & ~size_t(255);
-    return b;
+// Backward workspace: fp32 accumulators dQ [hq][T][d] (head-major), dK and dV
+// [T][hkv][d]
+// (one contiguous, 256-byte aligned block, cleared by one memset), then D
+// [hq][T] when the caller does not pass it.
+struct BwdWs {
+    size_t dq, dk, dv, acc_end, D, total;
+};
+inline size_t al256(size_t b) { return (b + 255) & ~size_t(255); }
+BwdWs bwd_ws_layout(const lf_attn_desc* d, bool need_D) {
+    BwdWs w{};
+    w.dq = 0;
+    w.dk = al256((size_t)d->total_tokens * d->hq * d->d * sizeof(float));
+    w.dv = w.dk + al256((size_t)d->total_tokens * d->hkv * d->d * sizeof(float));
+    w.acc_end = w.dv + al256((size_t)d->total_tokens * d->hkv * d->d * sizeof(float));
+    w.D = w.acc_end;
+    w.total = w.acc_end + (need_D ? al256((size_t)d->total_tokens * d->hq * sizeof(float)) : 0);
+    return w;
 }
+size_t bwd_ws_bytes(const lf_attn_desc* d, bool need_D) { return bwd_ws_layout(d, need_D).total; }
 
 // [T][H][d] bf16 -> 3-D map (d, H, T), 64 x 1 x 128 boxes, 128-byte swizzle.
 bool make_thd_map(CUtensorMap* m, const void* base, int T, int H, int D) {
@@ -125,30 +138,19 @@ template <int D>
 lf_status launch_bwd(const lf_attn_desc* d, const void* q, const void* k, const void* v,
                      const float* lse, const void* dout, const float* Dv, const float* w,
                      const int32_t* kidx, const int32_t* kcnt, void* dq, void* dk, void* dv,
-                     float* dq_acc, cudaStream_t st) {
+                     void* ws, cudaStream_t st) {
     CUtensorMap mq, mk, mv, mdo;
     if (!make_thd_map(&mq, q, d->total_tokens, d->hq, D) ||
         !make_thd_map(&mk, k, d->total_tokens, d->hkv, D) ||
         !make_thd_map(&mv, v, d->total_tokens, d->hkv, D) ||
         !make_thd_map(&mdo, dout, d->total_tokens, d->hq, D))
         return LF_ERR_CUDA;
-    // fp32 accumulator [T][hq][D] as a 3-D map (D, hq, T) with 32-row boxes: the
-    // backward adds staged dQ tiles into it by TMA reduction
-    CUtensorMap mdq;
-    {
-        EncodeTiledFn enc = encode_tiled();
-        if (!enc) return LF_ERR_CUDA;
-        const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)d->hq, (cuuint64_t)d->total_tokens};
-        const cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)d->hq * D * 4};
-        const cuuint32_t box[3] = {(cuuint32_t)D, 1, 32};
-        const cuuint32_t estr[3] = {1, 1, 1};
-        if (enc(&mdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, dq_acc, dims, strides, box, estr,
-                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
-                CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-            return LF_ERR_CUDA;
-    }
-    const size_t nacc = (size_t)d->total_tokens * d->hq * D;
-    if (cudaMemsetAsync(dq_acc, 0, nacc * sizeof(float), st) != cudaSuccess) return LF_ERR_CUDA;
+    const BwdWs lay = bwd_ws_layout(d, false);
+    uint8_t* base = static_cast<uint8_t*>(ws);
+    float* dq_acc = reinterpret_cast<float*>(base + lay.dq);
+    float* dk_acc = reinterpret_cast<float*>(base + lay.dk);
+    float* dv_acc = reinterpret_cast<float*>(base + lay.dv);
+    if (cudaMemsetAsync(base, 0, lay.acc_end, st) != cudaSuccess) return LF_ERR_CUDA;
     lf::BwdParams p{};
     p.cu_seqlens = d->cu_seqlens;
     p.T = d->total_tokens;
@@ -166,19 +168,26 @@ lf_status launch_bwd(const lf_attn_desc* d, const void* q, const void* k, const 
     p.kept_idx = kidx;
     p.kept_cnt = kcnt;
     p.dq_acc = dq_acc;
-    p.dk = static_cast<__nv_bfloat16*>(dk);
-    p.dv = static_cast<__nv_bfloat16*>(dv);
+    p.dk_acc = dk_acc;
+    p.dv_acc = dv_acc;
     const uint32_t smem = lf::BwdSmem<D>::kAlloc;
     if (cudaFuncSetAttribute(lf::attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem) != cudaSuccess)
         return LF_ERR_CUDA;
-    dim3 grid(ntiles_of(d), d->hkv, d->nseq);
-    lf::attn_bwd_kernel<D><<<grid, lf::kBwdThreads, smem, st>>>(mq, mk, mv, mdo, mdq, p);
+    dim3 grid(ntiles_of(d), d->hq, d->nseq);
+    lf::attn_bwd_kernel<D><<<grid, lf::kBwdThreads, smem, st>>>(mq, mk, mv, mdo, p);
     if (launch_status() != LF_OK) return LF_ERR_CUDA;
-    const size_t n8 = nacc / 8;
-    const int blocks = (int)std::min<size_t>((n8 + 255) / 256, 148 * 16);
-    lf::dq_convert_kernel<<<blocks, 256, 0, st>>>(reinterpret_cast<const float4*>(dq_acc),
-                                                  static_cast<uint4*>(dq), n8, d->softmax_scale);
+    // fp32 accumulators -> bf16 results (dQ and dK take the softmax scale)
+    const size_t nq8 = (size_t)d->total_tokens * d->hq * D / 8;
+    const size_t nkv8 = (size_t)d->total_tokens * d->hkv * D / 8;
+    const int bq = (int)std::min<size_t>((nq8 + 255) / 256, 148 * 16);
+    const int bkv = (int)std::min<size_t>((nkv8 + 255) / 256, 148 * 16);
+    lf::acc_hmajor_to_thd_kernel<<<bq, 256, 0, st>>>(dq_acc, static_cast<uint4*>(dq),
+                                                     d->total_tokens, d->hq, D, d->softmax_scale);
+    lf::dq_convert_kernel<<<bkv, 256, 0, st>>>(reinterpret_cast<const float4*>(dk_acc),
+                                               static_cast<uint4*>(dk), nkv8, d->softmax_scale);
+    lf::dq_convert_kernel<<<bkv, 256, 0, st>>>(reinterpret_cast<const float4*>(dv_acc),
+                                               static_cast<uint4*>(dv), nkv8, 1.0f);
     return launch_status();
 }
 
@@ -310,21 +319,18 @@ lf_status lf_attn_bwd(const lf_attn_desc* desc, const void* q, const void* k, co
     if (desc->total_tokens == 0 || desc->max_seqlen == 0) return LF_OK;
     if (!ws || ws_bytes < bwd_ws_bytes(desc, D == nullptr)) return LF_ERR_WORKSPACE;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    float* dq_acc = static_cast<float*>(ws);
     const float* Dv = D;
     if (!Dv) {
-        const size_t acc = ((size_t)desc->total_tokens * desc->hq * desc->d * sizeof(float) + 255) &
-                           ~size_t(255);
-        float* Dw = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + acc);
+        float* Dw = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + bwd_ws_layout(desc, true).D);
         st = desc->d == 128 ? launch_norms<128>(desc, dout, o, nullptr, Dw, 0, s)
                             : launch_norms<64>(desc, dout, o, nullptr, Dw, 0, s);
         if (st != LF_OK) return st;
         Dv = Dw;
     }
     return desc->d == 128 ? launch_bwd<128>(desc, q, k, v, lse, dout, Dv, block_weight, kept_idx,
-                                            kept_cnt, dq, dk, dv, dq_acc, s)
+                                            kept_cnt, dq, dk, dv, ws, s)
                           : launch_bwd<64>(desc, q, k, v, lse, dout, Dv, block_weight, kept_idx,
-                                           kept_cnt, dq, dk, dv, dq_acc, s);
+                                           kept_cnt, dq, dk, dv, ws, s);
 }
 
 lf_status lf_attn_bwd_static_ws(const lf_attn_desc* desc, const void* q, const void* k,
@@ -349,22 +355,19 @@ lf_status lf_attn_bwd_static_ws(const lf_attn_desc* desc, const void* q, const v
     st = static_ws_address(&ws);
     if (st != LF_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    float* dq_acc = static_cast<float*>(ws);
     const float* Dv = D;
     if (!Dv) {
-        const size_t acc = ((size_t)desc->total_tokens * desc->hq * desc->d * sizeof(float) + 255) &
-                           ~size_t(255);
-        float* Dw = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + acc);
+        float* Dw = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + bwd_ws_layout(desc, true).D);
         st = desc->d == 128 ? launch_norms<128>(desc, dout, o, nullptr, Dw, 0, s)
                             : launch_norms<64>(desc, dout, o, nullptr, Dw, 0, s);
         if (st != LF_OK) return st;
         Dv = Dw;
     }
-    // launch_bwd clears the accumulator (cudaMemsetAsync) before the kernel
+    // launch_bwd clears the accumulators (cudaMemsetAsync) before the kernel
     return desc->d == 128 ? launch_bwd<128>(desc, q, k, v, lse, dout, Dv, block_weight, kept_idx,
-                                            kept_cnt, dq, dk, dv, dq_acc, s)
+                                            kept_cnt, dq, dk, dv, ws, s)
                           : launch_bwd<64>(desc, q, k, v, lse, dout, Dv, block_weight, kept_idx,
-                                           kept_cnt, dq, dk, dv, dq_acc, s);
+                                           kept_cnt, dq, dk, dv, ws, s);
 }
 
 lf_status lf_check_device_error(lf_stream_t stream) {

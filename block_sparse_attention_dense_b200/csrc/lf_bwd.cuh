@@ -4,24 +4,27 @@
 // only kept query blocks are loaded and computed, and their output gradient
 // carries the weight 1/p).
 //
-// One CTA owns a 128-row KV tile j of one KV head g of one segment and walks,
-// for every query head of g's group, the kept query tiles t (t >= j when
-// causal) from the compacted kept-block lists.  Each 128-row query tile is
-// handled as two 64-column halves so that the element-wise work on one half
-// overlaps the tensor-core work on the other.  Per half:
+// One CTA owns a 128-row KV tile j of one segment for ONE query head h and
+// walks the kept query tiles t of h (t >= j when causal) from the compacted
+// kept-block list.  CTAs are ordered KV tile fastest, so the CTAs resident at
+// any time share one head: that head's Q, dO and fp32 dQ accumulator stay in
+// L2, where the dQ reductions run at L2 rather than HBM speed.  The GQA sum over
+// the heads of a KV head is done by fp32 reductions of each CTA's dK/dV tile
+// (one per CTA, not per pair).  Each 128-row query tile is handled as two
+// 64-column halves, one per element-wise warpgroup, so that the element-wise
+// work on one half overlaps the tensor-core work on the other.  Per half:
 //   tcgen05 (SS): S^T  = K_j Q_h^T,  dP^T = V_j dO_h^T        (TMEM, fp32)
 //   element-wise: P = exp2(S*scale*log2e - LSE*log2e), dS = P (dP - D), both
 //                 times the block weight; P^T and dS^T rounded to bf16 back
 //                 into TMEM (over S^T / dP^T) and dS^T into shared memory
-//   tcgen05 (TS): dV_j += P^T dO_h, dK_j += dS^T Q_h   (A from TMEM; dK/dV
-//                 accumulate in TMEM over the whole walk: no atomics)
+//   tcgen05 (TS): dV_j += P^T dO_h, dK_j += dS^T Q_h   (A from TMEM)
 //   tcgen05 (SS): dQ_h^T = K_j^T dS^T_h                  (TMEM, lanes = d)
 //   dQ drain:     lane d adds column q of dQ_h^T into the fp32 accumulator;
 //                 a warp's 32 lanes hit 32 consecutive floats of one row.
-// Roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer, warps 4-7
-// element-wise + epilogue (thread = KV row = TMEM lane), warps 8-11 dQ drain
-// (thread = head-dim index = TMEM lane).  The epilogue writes dK (times
-// softmax_scale) and dV as bf16; a KV tile that no kept block reaches gets 0.
+// Roles (512 threads): warp 0 TMA producer and work list, warp 1 MMA issuer,
+// warps 4-7 element-wise half 0 (+ dV epilogue), warps 12-15 element-wise
+// half 1 (+ dK epilogue): thread = KV row = TMEM lane; warps 8-11 dQ drain
+// (thread = head-dim index = TMEM lane).
 //
 // Tensor memory (512 columns): dV [0,128) dK [128,256); half 0: S^T/P^T/dQ^T
 // [256,320), dP^T/dS^T [320,384); half 1: [384,448), [448,512).  Reuse of a
@@ -42,9 +45,9 @@ struct BwdParams {
     const float* block_weight; // [nseq][hq][nbmax]
     const int32_t* kept_idx;   // [nseq][hq][nbmax]
     const int32_t* kept_cnt;   // [nseq][hq]
-    float* dq_acc;             // [T][hq][D] fp32, zeroed by the caller
-    __nv_bfloat16* dk;
-    __nv_bfloat16* dv;
+    float* dq_acc;             // [hq][T][D] fp32 (head-major), zeroed by the caller
+    float* dk_acc;             // [T][hkv][D] fp32 (unscaled), zeroed by the caller
+    float* dv_acc;             // [T][hkv][D] fp32, zeroed by the caller
 };
 
 template <int D>
@@ -62,7 +65,7 @@ struct BwdSmem {
     static constexpr uint32_t kAlloc = kBytes + 1024;
 };
 
-constexpr int kBwdThreads = 384;
+constexpr int kBwdThreads = 512;
 
 // One (query head, query tile) pair of a KV tile's walk, published by the
 // producer warp so that no other role reads the kept lists from global memory.
@@ -72,8 +75,8 @@ struct PairEntry {
     float w0, w1;   // block weights of the tile's two 64-row halves
 };
 
-// Walks the kept query tiles of one (segment, KV head) group in ascending order
-// of (head in group, tile).  Every role runs its own copy of the same walk.
+// Walks the kept query tiles of heads g*G .. g*G+G-1 of one segment in
+// ascending order of (head, tile) (the backward uses G = 1: one head).
 struct KeptTileWalk {
     const int32_t* kept_idx;
     const int32_t* kept_cnt;
@@ -142,7 +145,7 @@ template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const __grid_constant__ CUtensorMap tm_dq, BwdParams prm) {
+                    BwdParams prm) {
     using L = BwdSmem<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -162,15 +165,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     uint64_t* bar_entry = bars + 16;      // [4] work-list ring
     PairEntry* ring = reinterpret_cast<PairEntry*>(bars + 20);   // [4] x 16 B
 
-    // KV tile fastest: CTAs resident together share one KV head's group, so its
-    // Q/dO stay in L2; within a group the lowest tiles (most work) start first
+    // KV tile fastest: CTAs resident together share one query head, so its Q,
+    // dO and dQ accumulator stay in L2; the lowest tiles (most work) start first
     const int jt = blockIdx.x;
-    const int g = blockIdx.y;
+    const int hq_ = blockIdx.y;             // query head
     const int s = blockIdx.z;
     int seg0, len;
     if (!load_segment(prm.cu_seqlens, s, prm.T, prm.max_seqlen, seg0, len, 30)) return;
     if (jt * 128 >= len) return;
-    const int G = prm.hq / prm.hkv;
+    const int g = hq_ / (prm.hq / prm.hkv); // its KV head
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t s_base = smem_addr(smem);
@@ -193,7 +196,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
         prefetch_tensormap(&tm_do);
-        prefetch_tensormap(&tm_dq);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, 512);
@@ -209,7 +211,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
     // Does this KV tile have any work?  (every role sees the same answer)
     KeptTileWalk walk;
-    walk.init(prm, G, g, s, jt, len);
+    walk.init(prm, 1, hq_, s, jt, len);
     const bool any = walk.next(true);
 
     constexpr uint32_t kIdescS = idesc_bf16(128, 64, 0, 0);    // S^T, dP^T halves
@@ -346,17 +348,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_wait(bar_done, 0, 37);
         }
         __syncwarp();
-    } else if (warp >= 4 && warp < 8) {
-        // ===================== element-wise (thread = KV row) =====================
-        const int r = tid - 128;                          // TMEM lane / KV row
+    } else if ((warp >= 4 && warp < 8) || warp >= 12) {
+        // ============ element-wise, one warpgroup per half (thread = KV row) ============
+        const int hf = warp >= 12 ? 1 : 0;                // the half this warpgroup owns
+        const int bar_id = hf ? 3 : 1;
+        const int r = (warp & 3) * 32 + lane;             // TMEM lane / KV row
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const int kv_local = jt * 128 + r;
         const bool kv_valid = kv_local < len;
+        const uint32_t t_s = tmem + 256 + hf * 128 + lane_off, t_dp = t_s + 64;
+        const uint32_t dsa = s_base + L::kDS + hf * L::kHalfDS;
         int n = 0;
         bool more = any, failed = false;
         for (;;) {
-            // uniform decision of the four warps; also: all are done with the old vectors
-            if (named_bar_or(1, 128, !more || failed)) break;
+            // uniform decision of the warpgroup; also: all are done with the old vectors
+            if (named_bar_or(bar_id, 128, !more || failed)) break;
             const bool got_e = mbar_wait_or_abort(&bar_entry[n & 3], (n >> 2) & 1, 41, abort_flag);
             const PairEntry e = ring[n & 3];
             if (!got_e || e.h < 0) {
@@ -364,117 +370,101 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 failed = !got_e;
                 continue;
             }
-            const int h = e.h, qt = e.tile, q0 = qt * 128;
-            {
-                const int q_local = q0 + r;
+            const int qt = e.tile, q0 = qt * 128;
+            if (r < 64) {
+                const int col = hf * 64 + r;
+                const int q_local = q0 + col;
                 float l2 = INFINITY, dd = 0.f;    // exp2(S - inf) = 0: columns past the segment vanish
                 if (q_local < len) {
-                    const size_t idx = (size_t)h * prm.T + seg0 + q_local;
+                    const size_t idx = (size_t)e.h * prm.T + seg0 + q_local;
                     l2 = prm.lse[idx] * 1.4426950408889634f;
                     dd = prm.Dvec[idx];
                 }
-                lse2_s[r] = l2;
-                dvec_s[r] = dd;
+                lse2_s[col] = l2;
+                dvec_s[col] = dd;
             }
-            named_bar_sync(1, 128);
+            named_bar_sync(bar_id, 128);
             const bool diag = prm.causal && qt == jt;
-            for (int hf = 0; hf < 2 && !failed; ++hf) {
-                const float w = kv_valid ? (hf ? e.w1 : e.w0) : 0.f;
-                const bool got = mbar_wait_or_abort(&bar_s_full[hf], n & 1, 38, abort_flag);
-                if (!__all_sync(0xffffffffu, got)) { failed = true; break; }
-                tc_fence_after();
-                const uint32_t t_s = tmem + 256 + hf * 128 + lane_off, t_dp = t_s + 64;
-                const uint32_t dsa = s_base + L::kDS + hf * L::kHalfDS;
-                // 16-column chunks; the next chunk's TMEM loads overlap this chunk's math
-                auto chunk = [&](int c, const uint32_t (&sr)[16], const uint32_t (&dr)[16]) {
-                    uint32_t pk[8], dk_[8];
+            const float w = kv_valid ? (hf ? e.w1 : e.w0) : 0.f;
+            const bool got = mbar_wait_or_abort(&bar_s_full[hf], n & 1, 38, abort_flag);
+            if (!__all_sync(0xffffffffu, got)) { failed = true; continue; }
+            tc_fence_after();
+            // 16-column chunks; the next chunk's TMEM loads overlap this chunk's math
+            auto chunk = [&](int c, const uint32_t (&sr)[16], const uint32_t (&dr)[16]) {
+                uint32_t pk[8], dk_[8];
 #pragma unroll
-                    for (int e4 = 0; e4 < 4; ++e4) {
-                        const int col0 = hf * 64 + c * 16 + 4 * e4;
-                        const float4 l4 = *reinterpret_cast<const float4*>(lse2_s + col0);
-                        const float4 d4 = *reinterpret_cast<const float4*>(dvec_s + col0);
-                        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-                        const float dv_[4] = {d4.x, d4.y, d4.z, d4.w};
-                        float pw[4], dsw[4];
+                for (int e4 = 0; e4 < 4; ++e4) {
+                    const int col0 = hf * 64 + c * 16 + 4 * e4;
+                    const float4 l4 = *reinterpret_cast<const float4*>(lse2_s + col0);
+                    const float4 d4 = *reinterpret_cast<const float4*>(dvec_s + col0);
+                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                    const float dv_[4] = {d4.x, d4.y, d4.z, d4.w};
+                    float pw[4], dsw[4];
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            float p = fast_exp2(fmaf(__uint_as_float(sr[4 * e4 + u]), prm.scale_log2, -lv[u]));
-                            if (diag && kv_local > q0 + col0 + u) p = 0.f;
-                            pw[u] = p * w;
-                            dsw[u] = pw[u] * (__uint_as_float(dr[4 * e4 + u]) - dv_[u]);
-                        }
-                        pk[2 * e4] = pack_bf16(pw[0], pw[1]);
-                        pk[2 * e4 + 1] = pack_bf16(pw[2], pw[3]);
-                        dk_[2 * e4] = pack_bf16(dsw[0], dsw[1]);
-                        dk_[2 * e4 + 1] = pack_bf16(dsw[2], dsw[3]);
+                    for (int u = 0; u < 4; ++u) {
+                        float p = fast_exp2(fmaf(__uint_as_float(sr[4 * e4 + u]), prm.scale_log2, -lv[u]));
+                        if (diag && kv_local > q0 + col0 + u) p = 0.f;
+                        pw[u] = p * w;
+                        dsw[u] = pw[u] * (__uint_as_float(dr[4 * e4 + u]) - dv_[u]);
                     }
-                    // P^T over S^T (packed columns [8c, 8c+8)), dS^T over dP^T: columns
-                    // whose fp32 values were read by earlier chunks
-                    tmem_st8(t_s + c * 8, pk);
-                    tmem_st8(t_dp + c * 8, dk_);
-                    // dS^T into shared memory (one 64-column panel, SW128)
-                    st_shared_v4(dsa + sw128_chunk_offset(r, 2 * c), dk_[0], dk_[1], dk_[2], dk_[3]);
-                    st_shared_v4(dsa + sw128_chunk_offset(r, 2 * c + 1), dk_[4], dk_[5], dk_[6], dk_[7]);
-                };
-                uint32_t sa[16], da[16], sb[16], db[16];
-                tmem_ld16_nowait(t_s, sa);
-                tmem_ld16_nowait(t_dp, da);
-                tmem_wait_ld_regs(sa, da);
-                tmem_ld16_nowait(t_s + 16, sb);
-                tmem_ld16_nowait(t_dp + 16, db);
-                chunk(0, sa, da);
-                tmem_wait_ld_regs(sb, db);
-                tmem_ld16_nowait(t_s + 32, sa);
-                tmem_ld16_nowait(t_dp + 32, da);
-                chunk(1, sb, db);
-                tmem_wait_ld_regs(sa, da);
-                tmem_ld16_nowait(t_s + 48, sb);
-                tmem_ld16_nowait(t_dp + 48, db);
-                chunk(2, sa, da);
-                tmem_wait_ld_regs(sb, db);
-                chunk(3, sb, db);
-                tmem_wait_st();
-                fence_proxy_async_smem();
-                tc_fence_before();
-                mbar_arrive(&bar_p_ready[hf]);
-            }
-            if (!failed) ++n;
+                    pk[2 * e4] = pack_bf16(pw[0], pw[1]);
+                    pk[2 * e4 + 1] = pack_bf16(pw[2], pw[3]);
+                    dk_[2 * e4] = pack_bf16(dsw[0], dsw[1]);
+                    dk_[2 * e4 + 1] = pack_bf16(dsw[2], dsw[3]);
+                }
+                // P^T over S^T (packed columns [8c, 8c+8)), dS^T over dP^T: columns
+                // whose fp32 values were read by earlier chunks
+                tmem_st8(t_s + c * 8, pk);
+                tmem_st8(t_dp + c * 8, dk_);
+                // dS^T into shared memory (one 64-column panel, SW128)
+                st_shared_v4(dsa + sw128_chunk_offset(r, 2 * c), dk_[0], dk_[1], dk_[2], dk_[3]);
+                st_shared_v4(dsa + sw128_chunk_offset(r, 2 * c + 1), dk_[4], dk_[5], dk_[6], dk_[7]);
+            };
+            uint32_t sa[16], da[16], sb[16], db[16];
+            tmem_ld16_nowait(t_s, sa);
+            tmem_ld16_nowait(t_dp, da);
+            tmem_wait_ld_regs(sa, da);
+            tmem_ld16_nowait(t_s + 16, sb);
+            tmem_ld16_nowait(t_dp + 16, db);
+            chunk(0, sa, da);
+            tmem_wait_ld_regs(sb, db);
+            tmem_ld16_nowait(t_s + 32, sa);
+            tmem_ld16_nowait(t_dp + 32, da);
+            chunk(1, sb, db);
+            tmem_wait_ld_regs(sa, da);
+            tmem_ld16_nowait(t_s + 48, sb);
+            tmem_ld16_nowait(t_dp + 48, db);
+            chunk(2, sa, da);
+            tmem_wait_ld_regs(sb, db);
+            chunk(3, sb, db);
+            tmem_wait_st();
+            fence_proxy_async_smem();
+            tc_fence_before();
+            mbar_arrive(&bar_p_ready[hf]);
+            ++n;
         }
-        // ---- epilogue: dV, dK (x softmax_scale) for this thread's KV row ----
+        // ---- epilogue: warpgroup 0 adds dV, warpgroup 1 adds dK (unscaled) into the
+        // fp32 accumulators of the KV head (the GQA sum over query heads) ----
         bool have = n > 0 && !failed && !*abort_flag;
         if (have) have = mbar_wait_or_abort(bar_done, 0, 39, abort_flag);
         have = __all_sync(0xffffffffu, have);
-        tc_fence_after();
-        const bool write = kv_valid && (have || (n == 0 && !failed));
-        const size_t orow = ((size_t)(kv_row0 + r) * prm.hkv + g) * D;
+        if (have) {
+            tc_fence_after();
+            float* dst = (hf ? prm.dk_acc : prm.dv_acc) + ((size_t)(kv_row0 + r) * prm.hkv + g) * D;
+            const uint32_t t_acc = (hf ? t_dk : t_dv) + lane_off;
 #pragma unroll 1
-        for (int c = 0; c < D / 32; ++c) {
-            float v[32], k[32];
-            if (have) {
-                tmem_ld32(t_dv + lane_off + c * 32, v);
-                tmem_ld32(t_dk + lane_off + c * 32, k);
-            } else {
+            for (int c = 0; c < D / 32; ++c) {
+                float v[32];
+                tmem_ld32(t_acc + c * 32, v);
+                if (kv_valid) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) { v[e] = 0.f; k[e] = 0.f; }
-            }
-            if (write) {
-#pragma unroll
-                for (int e8 = 0; e8 < 4; ++e8) {
-                    uint4 pv, pk;
-                    pv.x = pack_bf16(v[e8 * 8 + 0], v[e8 * 8 + 1]);
-                    pv.y = pack_bf16(v[e8 * 8 + 2], v[e8 * 8 + 3]);
-                    pv.z = pack_bf16(v[e8 * 8 + 4], v[e8 * 8 + 5]);
-                    pv.w = pack_bf16(v[e8 * 8 + 6], v[e8 * 8 + 7]);
-                    pk.x = pack_bf16(k[e8 * 8 + 0] * prm.scale, k[e8 * 8 + 1] * prm.scale);
-                    pk.y = pack_bf16(k[e8 * 8 + 2] * prm.scale, k[e8 * 8 + 3] * prm.scale);
-                    pk.z = pack_bf16(k[e8 * 8 + 4] * prm.scale, k[e8 * 8 + 5] * prm.scale);
-                    pk.w = pack_bf16(k[e8 * 8 + 6] * prm.scale, k[e8 * 8 + 7] * prm.scale);
-                    *reinterpret_cast<uint4*>(prm.dv + orow + c * 32 + e8 * 8) = pv;
-                    *reinterpret_cast<uint4*>(prm.dk + orow + c * 32 + e8 * 8) = pk;
+                    for (int e4 = 0; e4 < 8; ++e4)
+                        atomicAdd(reinterpret_cast<float4*>(dst + c * 32 + 4 * e4),
+                                  make_float4(v[4 * e4], v[4 * e4 + 1], v[4 * e4 + 2], v[4 * e4 + 3]));
                 }
             }
         }
-    } else if (warp >= 8) {
+    } else if (warp >= 8 && warp < 12) {
         // ===================== dQ drain (thread = head-dim index) =====================
         const int dd = tid - 256;                         // TMEM lane = d index
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
@@ -486,37 +476,26 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!__all_sync(0xffffffffu, got_e)) break;
             const PairEntry e = ring[n & 3];
             if (e.h < 0) break;
-            const int h = e.h, q0 = e.tile * 128;
+            const int q0 = e.tile * 128;
             bool ok = true;
             for (int hf = 0; hf < 2; ++hf) {
                 const bool got = mbar_wait_or_abort(&bar_dq_full[hf], n & 1, 40, abort_flag);
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
                 tc_fence_after();
                 const int qh = q0 + hf * 64;
-                const bool live = qh < len && (hf ? e.w1 : e.w0) != 0.f;
+                const bool live = lane_used && qh < len && (hf ? e.w1 : e.w0) != 0.f;
                 if (live) {
-                    // The half's dS^T buffer is idle from the end of its dQ^T MMA until
-                    // dq_free: stage 32 query rows x d fp32 there and let TMA add them
-                    // into the accumulator (rows past T are clipped by TMA; rows past
-                    // the segment carry exact zeros).
-                    float* stage = reinterpret_cast<float*>(smem + L::kDS + hf * L::kHalfDS);
                     const uint32_t t_q = tmem + 256 + hf * 128 + lane_off;
-                    for (int rnd = 0; rnd < 2; ++rnd) {
-                        if (qh + rnd * 32 >= len) break;
-                        if (lane_used) {
-                            float v[32];
-                            tmem_ld32(t_q + rnd * 32, v);
+                    // head-major accumulator: the half's 64 query rows are contiguous
+                    float* dst = prm.dq_acc + ((size_t)e.h * prm.T + seg0 + qh) * D + dd;
+                    const int nvalid = min(64, len - qh);
 #pragma unroll
-                            for (int q = 0; q < 32; ++q) stage[q * D + dd] = v[q];
-                        }
-                        fence_proxy_async_smem();
-                        named_bar_sync(2, 128);
-                        if (dd == 0) {
-                            tma_reduce_add_3d(&tm_dq, stage, 0, h, seg0 + qh + rnd * 32);
-                            bulk_commit_group();
-                            bulk_wait_read0();
-                        }
-                        named_bar_sync(2, 128);   // the stage may be written again
+                    for (int c = 0; c < 2; ++c) {
+                        float v[32];
+                        tmem_ld32(t_q + c * 32, v);
+#pragma unroll
+                        for (int q = 0; q < 32; ++q)
+                            if (c * 32 + q < nvalid) atomicAdd(dst + (c * 32 + q) * D, v[q]);
                     }
                 }
                 tc_fence_before();
@@ -525,7 +504,6 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!ok) break;
             ++n;
         }
-        if (dd == 0) bulk_wait0();   // reductions performed before the CTA retires
     }
 
     tc_fence_before();

@@ -205,4 +205,30 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const float4* __restric
     }
 }
 
+// ---------------------------------------------------------------------------
+// dQ = scale * accumulator with the head-major accumulator [H][T][D] permuted
+// to the THD output [T][H][D]; one thread converts 8 consecutive d.
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) acc_hmajor_to_thd_kernel(const float* __restrict__ acc,
+                                                                uint4* __restrict__ out, int T,
+                                                                int H, int D, float scale) {
+    const int d8 = D / 8;
+    const size_t n8 = (size_t)T * H * d8;
+    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8;
+         i += (size_t)gridDim.x * blockDim.x) {
+        const int c = (int)(i % d8);
+        const size_t th = i / d8;                 // t * H + h
+        const int h = (int)(th % H);
+        const size_t t = th / H;
+        const float4* src = reinterpret_cast<const float4*>(acc + ((size_t)h * T + t) * D + c * 8);
+        const float4 a = src[0], b = src[1];
+        uint4 r;
+        r.x = pack_bf16(a.x * scale, a.y * scale);
+        r.y = pack_bf16(a.z * scale, a.w * scale);
+        r.z = pack_bf16(b.x * scale, b.y * scale);
+        r.w = pack_bf16(b.z * scale, b.w * scale);
+        out[i] = r;
+    }
+}
+
 }  // namespace lf

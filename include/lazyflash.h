@@ -142,17 +142,17 @@ lf_status lf_attn_bwd(const lf_attn_desc* desc, const void* q, const void* k, co
  * that plan all device memory ahead of time or forbid cudaMalloc/cudaFree while
  * they run (those calls synchronize the device and are not allowed inside a
  * stream capture).
- *   Arguments and results are those of lf_attn_bwd.  The scratch (the fp32 dQ
- *   accumulator, plus D when D is NULL) lives in one file-scope device array of
- *   LF_STATIC_WS_BYTES bytes that every GPU loading the library holds until the
- *   process exits.  A problem whose scratch exceeds it, i.e.
- *   4 * total_tokens * hq * d bytes (rounded up to 256), plus
- *   4 * total_tokens * hq when D is NULL, returns LF_ERR_WORKSPACE before
- *   anything is launched.
+ *   Arguments and results are those of lf_attn_bwd.  The scratch (the fp32
+ *   accumulators of dQ, dK and dV, plus D when D is NULL) lives in one
+ *   file-scope device array of LF_STATIC_WS_BYTES bytes that every GPU loading
+ *   the library holds until the process exits.  A problem whose scratch
+ *   exceeds it, i.e. 4 * total_tokens * (hq + 2 * hkv) * d bytes (each of the
+ *   three parts rounded up to 256), plus 4 * total_tokens * hq when D is NULL,
+ *   returns LF_ERR_WORKSPACE before anything is launched.
  *   The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current); make that first call
  *   before any stream capture.  The call never calls cudaMalloc, cudaFree or an
- *   allocating library routine; the accumulator is cleared at the start of
+ *   allocating library routine; the accumulators are cleared at the start of
  *   every call.
  *   All calls on a device share the one array and it keeps the last call's
  *   contents: calls that may overlap on the GPU (different streams, or host
