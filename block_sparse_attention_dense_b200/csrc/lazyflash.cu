@@ -118,7 +118,9 @@ lf_status launch_fwd(const lf_attn_desc* d, const void* q, const void* k, const 
     if (cudaFuncSetAttribute(lf::attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem) != cudaSuccess)
         return LF_ERR_CUDA;
-    dim3 grid(d->hq, ntiles_of(d), d->nseq);
+    // one CTA per pair of query tiles; pair index fastest so that the CTAs resident
+    // together share a head (its K/V stay in L2)
+    dim3 grid((ntiles_of(d) + 1) / 2, d->hq, d->nseq);
     lf::attn_fwd_kernel<D><<<grid, lf::kFwdThreads, smem, st>>>(mq, mk, mv, p);
     return launch_status();
 }

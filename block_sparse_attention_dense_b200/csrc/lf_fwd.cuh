@@ -2,15 +2,23 @@
 // unchanged: article standfirst and section "Le passage arrière fait deux fois
 // le travail du passage avant").
 //
-// One CTA computes a 128-row query tile of one head of one segment:
-//   TMA:      Q tile once, K/V tiles double-buffered (128 x d, SW128 panels);
-//   tcgen05:  S = Q K^T into TMEM (128 lanes x 128 fp32 columns),
-//             O += P V into TMEM (128 lanes x d columns);
-//   4 warps:  thread r owns query row r (TMEM lane r): online softmax in the
-//             exp2 domain, P rounded to bf16 into shared memory in the
-//             tensor core's K-major layout, O rescaled in TMEM when the row
-//             maximum moves;
-//   epilogue: O / l -> bf16, LSE = ln(l) + max (natural log).
+// One CTA computes two consecutive 128-row query tiles (2m, 2m+1) of one head
+// of one segment, in ping-pong: while one softmax warpgroup turns its score
+// tile into probabilities, the tensor core computes the other tile's scores
+// and P.V products.
+//   TMA:      both Q tiles once; K and V tiles through two-stage rings;
+//   tcgen05:  S_t = Q_t K_j^T (SS, 128 x 128 fp32 in TMEM), O_t += P_t V_j
+//             (TS: P_t read from TMEM, where the softmax wrote it over S_t);
+//   softmax:  warpgroup t, thread r owns query row r (TMEM lane r): online
+//             softmax in the exp2 domain with a stale-max rule (the reference
+//             maximum moves only when the row maximum grows by more than 2^8,
+//             and only then is O rescaled in TMEM);
+//   epilogue: O / l -> bf16, LSE = (m + log2 l) * ln 2.
+// Roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer, warps 4-7
+// softmax of tile 0, warps 8-11 softmax of tile 1.
+// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d),
+// O1 [384,384+d); P_t (bf16, packed two per column) over S_t [0,64).  Reuse
+// of a region by a later MMA relies on tcgen05.mma executing in issue order.
 #pragma once
 
 #include "lf_device.cuh"
@@ -29,16 +37,16 @@ template <int D>
 struct FwdSmem {
     static constexpr int kPanels = D / 64;
     static constexpr uint32_t kTile = kPanels * kPanelBytes;     // one 128 x D bf16 tile
-    static constexpr uint32_t kQ = 0;
-    static constexpr uint32_t kK = kQ + kTile;                   // 2 stages
+    static constexpr uint32_t kQ = 0;                            // 2 tiles
+    static constexpr uint32_t kK = kQ + 2 * kTile;               // 2 stages
     static constexpr uint32_t kV = kK + 2 * kTile;               // 2 stages
-    static constexpr uint32_t kP = kV + 2 * kTile;               // 128 x 128 bf16
-    static constexpr uint32_t kBars = kP + 2 * kPanelBytes;
-    static constexpr uint32_t kBytes = kBars + 64;
+    static constexpr uint32_t kBars = kV + 2 * kTile;
+    static constexpr uint32_t kBytes = kBars + 256;
     static constexpr uint32_t kAlloc = kBytes + 1024;            // slack for 1024-B alignment
 };
 
-constexpr int kFwdThreads = 128;
+constexpr int kFwdThreads = 384;
+constexpr float kRescaleThreshold = 8.0f;   // log2 of the largest P before a rescale
 
 template <int D>
 __global__ void __launch_bounds__(kFwdThreads, 1)
@@ -47,30 +55,49 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     using L = FwdSmem<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    uint64_t* bar_q = reinterpret_cast<uint64_t*>(smem + L::kBars);
-    uint64_t* bar_kv = bar_q + 1;     // [2]
-    uint64_t* bar_mma = bar_q + 3;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar_q + 4);
-    int* abort_flag = reinterpret_cast<int*>(bar_q + 5);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
+    uint64_t* bar_q = bars + 0;
+    uint64_t* bar_k_full = bars + 1;    // [2]
+    uint64_t* bar_k_empty = bars + 3;   // [2]
+    uint64_t* bar_v_full = bars + 5;    // [2]
+    uint64_t* bar_v_empty = bars + 7;   // [2]
+    uint64_t* bar_s_full = bars + 9;    // [2] per query tile
+    uint64_t* bar_p_ready = bars + 11;  // [2]
+    uint64_t* bar_o_done = bars + 13;   // [2]
+    uint64_t* bar_done = bars + 15;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 17);
 
-    const int h = blockIdx.x;
+    const int h = blockIdx.y;
     const int s = blockIdx.z;
     int seg0, len;
     if (!load_segment(prm.cu_seqlens, s, prm.T, prm.max_seqlen, seg0, len, 20)) return;
     const int ntiles = (len + 127) >> 7;
-    const int qt = ntiles - 1 - static_cast<int>(blockIdx.y);   // longest rows first
-    if (qt < 0) return;
+    const int npairs = (ntiles + 1) >> 1;
+    const int m = npairs - 1 - static_cast<int>(blockIdx.x);   // longest rows first
+    if (m < 0) return;
     const int g = h / (prm.hq / prm.hkv);
-    const int nkv = prm.causal ? qt + 1 : ntiles;
+    const bool two = 2 * m + 1 < ntiles;                     // tile 1 exists
+    // KV tiles each query tile needs
+    const int nkv0 = prm.causal ? 2 * m + 1 : ntiles;
+    const int nkv1 = two ? (prm.causal ? 2 * m + 2 : ntiles) : 0;
+    const int nkv = nkv0 > nkv1 ? nkv0 : nkv1;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t s_base = smem_addr(smem);
 
     if (tid == 0) {
         mbar_init(bar_q, 1);
-        mbar_init(&bar_kv[0], 1);
-        mbar_init(&bar_kv[1], 1);
-        mbar_init(bar_mma, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&bar_k_full[i], 1);
+            mbar_init(&bar_k_empty[i], 1);
+            mbar_init(&bar_v_full[i], 1);
+            mbar_init(&bar_v_empty[i], 1);
+            mbar_init(&bar_s_full[i], 1);
+            mbar_init(&bar_p_ready[i], 128);
+            mbar_init(&bar_o_done[i], 1);
+        }
+        mbar_init(bar_done, 1);
         *abort_flag = 0;
         fence_barrier_init();
         prefetch_tensormap(&tm_q);
@@ -78,181 +105,238 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         prefetch_tensormap(&tm_v);
     }
     if (warp == 0) {
-        tmem_alloc(tmem_slot, 256);
+        tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t t_s = tmem;            // S: columns [0, 128)
-    const uint32_t t_o = tmem + 128;      // O: columns [128, 128 + D)
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
 
-    const int row0 = seg0 + qt * 128;
-    if (tid == 0) {
-        mbar_arrive_expect_tx(bar_q, L::kTile);
-        for (int c = 0; c < L::kPanels; ++c)
-            tma_load_3d(smem + L::kQ + c * kPanelBytes, &tm_q, bar_q, c * 64, h, row0);
-        mbar_arrive_expect_tx(&bar_kv[0], 2 * L::kTile);
-        for (int c = 0; c < L::kPanels; ++c) {
-            tma_load_3d(smem + L::kK + c * kPanelBytes, &tm_k, &bar_kv[0], c * 64, g, seg0);
-            tma_load_3d(smem + L::kV + c * kPanelBytes, &tm_v, &bar_kv[0], c * 64, g, seg0);
-        }
-    }
-
-    constexpr uint32_t kIdescS = idesc_bf16(128, 128, 0, 0);
-    constexpr uint32_t kIdescO = idesc_bf16(128, D, 0, 1);
-    const int q_local = qt * 128 + tid;     // this thread's query row within the segment
-    float m_run = -INFINITY, l_run = 0.f;
-    uint32_t mma_phase = 0;
-    bool ok = true;
-    // loads issued / waited per K-V stage (thread 0 only), for the drain on abort
-    int kv_issued[2] = {1, 0}, kv_waited[2] = {0, 0};
-    bool q_waited = false;
-
-    for (int j = 0; j < nkv && ok; ++j) {
-        const int st = j & 1;
-        if (tid == 0) {
-            if (j + 1 < nkv) {
-                const int ns = st ^ 1;
-                mbar_arrive_expect_tx(&bar_kv[ns], 2 * L::kTile);
-                ++kv_issued[ns];
-                for (int c = 0; c < L::kPanels; ++c) {
-                    tma_load_3d(smem + L::kK + ns * L::kTile + c * kPanelBytes, &tm_k, &bar_kv[ns],
-                                c * 64, g, seg0 + (j + 1) * 128);
-                    tma_load_3d(smem + L::kV + ns * L::kTile + c * kPanelBytes, &tm_v, &bar_kv[ns],
-                                c * 64, g, seg0 + (j + 1) * 128);
+    if (warp == 0) {
+        // ===================== TMA producer =====================
+        if (lane == 0) {
+            const uint32_t qbytes = (two ? 2 : 1) * L::kTile;
+            mbar_arrive_expect_tx(bar_q, qbytes);
+            for (int t = 0; t < (two ? 2 : 1); ++t)
+                for (int c = 0; c < L::kPanels; ++c)
+                    tma_load_3d(smem + L::kQ + t * L::kTile + c * kPanelBytes, &tm_q, bar_q, c * 64, h,
+                                seg0 + (2 * m + t) * 128);
+            uint32_t kpar[2] = {0, 0}, vpar[2] = {0, 0};
+            int kfill = 0, vfill = 0;   // loads issued (for the drain on abort)
+            for (int j = 0; j < nkv; ++j) {
+                const int st = j & 1;
+                if (j >= 2 && !mbar_wait_or_abort(&bar_k_empty[st], ((j >> 1) - 1) & 1, 21, abort_flag)) break;
+                mbar_arrive_expect_tx(&bar_k_full[st], L::kTile);
+                for (int c = 0; c < L::kPanels; ++c)
+                    tma_load_3d(smem + L::kK + st * L::kTile + c * kPanelBytes, &tm_k, &bar_k_full[st],
+                                c * 64, g, seg0 + j * 128);
+                kpar[st] = (j >> 1) & 1;
+                ++kfill;
+                if (j >= 2 && !mbar_wait_or_abort(&bar_v_empty[st], ((j >> 1) - 1) & 1, 22, abort_flag)) break;
+                mbar_arrive_expect_tx(&bar_v_full[st], L::kTile);
+                for (int c = 0; c < L::kPanels; ++c)
+                    tma_load_3d(smem + L::kV + st * L::kTile + c * kPanelBytes, &tm_v, &bar_v_full[st],
+                                c * 64, g, seg0 + j * 128);
+                vpar[st] = (j >> 1) & 1;
+                ++vfill;
+            }
+            if (*abort_flag) {
+                // let this CTA's own copies land before the CTA exits (bounded)
+                mbar_wait(bar_q, 0, 23);
+                for (int st = 0; st < 2; ++st) {
+                    if (kfill > st) mbar_wait(&bar_k_full[st], kpar[st], 23);
+                    if (vfill > st) mbar_wait(&bar_v_full[st], vpar[st], 23);
                 }
             }
-            bool w_ok = q_waited || mbar_wait(bar_q, 0, 1);
-            q_waited = w_ok;
-            w_ok = w_ok && mbar_wait(&bar_kv[st], (j >> 1) & 1, 2);
-            if (w_ok) ++kv_waited[st];
-            if (w_ok) {
-                tc_fence_after();
-                const uint32_t qa = s_base + L::kQ;
-                const uint32_t ka = s_base + L::kK + st * L::kTile;
+        }
+        __syncwarp();
+    } else if (warp == 1) {
+        // ===================== MMA issuer (one thread) =====================
+        if (lane == 0) {
+            constexpr uint32_t kIdescS = idesc_bf16(128, 128, 0, 0);
+            constexpr uint32_t kIdescO = idesc_bf16(128, D, 0, 1);
+            const uint32_t qa0 = s_base + L::kQ;
+            auto issue_s = [&](int t, int j) {
+                const uint32_t qa = qa0 + t * L::kTile;
+                const uint32_t ka = s_base + L::kK + (j & 1) * L::kTile;
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k)
-                    mma_bf16_ss(t_s, desc_kmajor(qa, k), desc_kmajor(ka, k), kIdescS, k > 0);
-                mma_commit(bar_mma);
+                    mma_bf16_ss(tmem + t * 128, desc_kmajor(qa, k), desc_kmajor(ka, k), kIdescS, k > 0);
+                mma_commit(&bar_s_full[t]);
+            };
+            bool ok = mbar_wait_or_abort(bar_q, 0, 24, abort_flag) &&
+                      mbar_wait_or_abort(&bar_k_full[0], 0, 25, abort_flag);
+            if (ok) {
+                tc_fence_after();
+                issue_s(0, 0);
+                if (two) issue_s(1, 0);
+                mma_commit(&bar_k_empty[0]);
+            }
+            for (int j = 0; j < nkv && ok; ++j) {
+                const int st = j & 1;
+                if (!mbar_wait_or_abort(&bar_v_full[st], (j >> 1) & 1, 26, abort_flag)) break;
+                bool k_next_ready = false;
+                for (int t = 0; t < 2; ++t) {
+                    const int nk = t ? nkv1 : nkv0;
+                    if (j >= nk) continue;
+                    if (!mbar_wait_or_abort(&bar_p_ready[t], j & 1, 27, abort_flag)) { ok = false; break; }
+                    tc_fence_after();
+                    const uint32_t va = s_base + L::kV + st * L::kTile;
+#pragma unroll
+                    for (int k = 0; k < 8; ++k)
+                        mma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + k * 8, desc_mnmajor(va, k),
+                                    kIdescO, (j > 0 || k > 0) ? 1u : 0u);
+                    mma_commit(&bar_o_done[t]);
+                    if (j + 1 < nk) {
+                        if (!k_next_ready) {
+                            if (!mbar_wait_or_abort(&bar_k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, 28, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            tc_fence_after();
+                            k_next_ready = true;
+                        }
+                        issue_s(t, j + 1);
+                    }
+                }
+                if (!ok) break;
+                mma_commit(&bar_v_empty[st]);
+                if (k_next_ready) mma_commit(&bar_k_empty[(j + 1) & 1]);
+            }
+            mma_commit(bar_done);
+            mbar_wait(bar_done, 0, 29);   // every MMA issued here has finished
+        }
+        __syncwarp();
+    } else if (warp >= 4 && warp < 12) {
+        // ============ softmax, one warpgroup per query tile (thread = row) ============
+        const int t = (warp - 4) >> 2;
+        const int r = (warp & 3) * 32 + lane;
+        const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+        const uint32_t t_s = tmem + t * 128 + lane_off;
+        const uint32_t t_o = tmem + 256 + t * 128 + lane_off;
+        const int nk = t ? nkv1 : nkv0;
+        const int qt = 2 * m + t;
+        const int q_local = qt * 128 + r;
+        float m_ref = -INFINITY, l_run = 0.f;
+        bool failed = false;
+        for (int j = 0; j < nk; ++j) {
+            const bool got = mbar_wait_or_abort(&bar_s_full[t], j & 1, 30, abort_flag);
+            if (!__all_sync(0xffffffffu, got)) { failed = true; break; }
+            tc_fence_after();
+            float sv[128];
+            {
+                uint32_t a[16], b[16];
+#pragma unroll
+                for (int c = 0; c < 8; c += 2) {
+                    tmem_ld16_nowait(t_s + c * 16, a);
+                    tmem_ld16_nowait(t_s + (c + 1) * 16, b);
+                    tmem_wait_ld_regs(a, b);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        sv[c * 16 + e] = __uint_as_float(a[e]);
+                        sv[(c + 1) * 16 + e] = __uint_as_float(b[e]);
+                    }
+                }
+            }
+            const int kv0 = j * 128;
+            const bool diag = prm.causal && j == qt;
+            const bool tail = kv0 + 128 > len;
+            float mx = -INFINITY;
+            if (diag || tail) {
+#pragma unroll
+                for (int e = 0; e < 128; ++e) {
+                    const int kv = kv0 + e;
+                    const bool valid = !(diag && kv > q_local) && kv < len;
+                    sv[e] = valid ? sv[e] * prm.scale_log2 : -INFINITY;
+                    mx = fmaxf(mx, sv[e]);
+                }
             } else {
-                *abort_flag = 1;
+#pragma unroll
+                for (int e = 0; e < 128; ++e) {
+                    sv[e] *= prm.scale_log2;
+                    mx = fmaxf(mx, sv[e]);
+                }
             }
-        }
-        __syncthreads();
-        if (*abort_flag) { ok = false; break; }
-        if (!mbar_wait(bar_mma, mma_phase, 3)) *abort_flag = 1;
-        mma_phase ^= 1;
-        __syncthreads();
-        if (*abort_flag) { ok = false; break; }
-        tc_fence_after();
-
-        // ---- online softmax on this thread's row ----
-        float sv[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            float tmp[32];
-            tmem_ld32(t_s + lane_off + c * 32, tmp);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) sv[c * 32 + e] = tmp[e];
-        }
-        const int kv0 = j * 128;
-        const bool diag = prm.causal ? (kv0 + 127 > q_local) : false;
-        const bool tail = kv0 + 128 > len;
-        float mx = -INFINITY;
-#pragma unroll
-        for (int e = 0; e < 128; ++e) {
-            const int kv = kv0 + e;
-            const bool valid = !(diag && kv > q_local) && !(tail && kv >= len);
-            sv[e] = valid ? sv[e] * prm.scale_log2 : -INFINITY;
-            mx = fmaxf(mx, sv[e]);
-        }
-        const float m_new = fmaxf(m_run, mx);
-        const float alpha = (m_run == -INFINITY) ? 0.f : fast_exp2(m_run - m_new);
-        float rs = 0.f;
-        const uint32_t p_base = s_base + L::kP;
-#pragma unroll
-        for (int ch = 0; ch < 16; ++ch) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int e2 = 0; e2 < 4; ++e2) {
-                const float p0 = fast_exp2(sv[ch * 8 + 2 * e2] - m_new);
-                const float p1 = fast_exp2(sv[ch * 8 + 2 * e2 + 1] - m_new);
-                rs += p0 + p1;
-                pk[e2] = pack_bf16(p0, p1);
+            // stale-max rule: keep the old reference unless the row maximum grew a lot
+            float alpha = 1.f;
+            bool rescale = false;
+            if (j == 0) {
+                m_ref = mx;
+            } else if (mx > m_ref + kRescaleThreshold) {
+                alpha = fast_exp2(m_ref - mx);
+                m_ref = mx;
+                rescale = true;
             }
-            st_shared_v4(p_base + sw128_chunk_offset(tid, ch), pk[0], pk[1], pk[2], pk[3]);
+            float rs = 0.f;
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const float p0 = fast_exp2(sv[c * 32 + 2 * e] - m_ref);
+                    const float p1 = fast_exp2(sv[c * 32 + 2 * e + 1] - m_ref);
+                    rs += p0 + p1;
+                    pk[e] = pack_bf16(p0, p1);
+                }
+                tmem_st16(t_s + c * 16, pk);   // P (packed) over S columns already read
+            }
+            l_run = l_run * alpha + rs;
+            if (__any_sync(0xffffffffu, rescale)) {
+                // O_t must hold the previous P.V product before it is rescaled
+                const bool got_o = mbar_wait_or_abort(&bar_o_done[t], (j - 1) & 1, 31, abort_flag);
+                if (!__all_sync(0xffffffffu, got_o)) { failed = true; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    float ov[32];
+                    tmem_ld32(t_o + c * 32, ov);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+                    tmem_st32(t_o + c * 32, ov);
+                }
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            mbar_arrive(&bar_p_ready[t]);
         }
-        l_run = l_run * alpha + rs;
-        m_run = m_new;
-        // rescale the running O when this row's maximum moved
-        if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        // ---- epilogue: O / l -> bf16, LSE ----
+        bool have = !failed && nk > 0 && !*abort_flag;
+        if (have) have = mbar_wait_or_abort(&bar_o_done[t], (nk - 1) & 1, 32, abort_flag);
+        have = __all_sync(0xffffffffu, have);
+        if (have) {
+            tc_fence_after();
+            const bool row_ok = q_local < len;
+            const float inv_l = 1.f / l_run;
+            const int tok = seg0 + q_local;
+            __nv_bfloat16* orow = prm.o + ((size_t)tok * prm.hq + h) * D;
 #pragma unroll
             for (int c = 0; c < D / 32; ++c) {
                 float ov[32];
-                tmem_ld32(t_o + lane_off + c * 32, ov);
+                tmem_ld32(t_o + c * 32, ov);
+                if (row_ok) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) ov[e] *= alpha;
-                tmem_st32(t_o + lane_off + c * 32, ov);
-            }
-            tmem_wait_st();
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t va = s_base + L::kV + st * L::kTile;
-#pragma unroll
-            for (int k = 0; k < 8; ++k)
-                mma_bf16_ss(t_o, desc_kmajor(p_base, k), desc_mnmajor(va, k), kIdescO,
-                            (j > 0 || k > 0) ? 1u : 0u);
-            mma_commit(bar_mma);
-        }
-        if (!mbar_wait(bar_mma, mma_phase, 4)) *abort_flag = 1;
-        mma_phase ^= 1;
-        __syncthreads();
-        if (*abort_flag) { ok = false; break; }
-        tc_fence_after();
-    }
-
-    if (ok) {
-        // ---- epilogue: O / l -> bf16, LSE ----
-        const bool row_ok = q_local < len;
-        const float inv_l = 1.f / l_run;
-        const int t = seg0 + q_local;
-        __nv_bfloat16* orow = prm.o + ((size_t)t * prm.hq + h) * D;
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
-            float ov[32];
-            tmem_ld32(t_o + lane_off + c * 32, ov);
-            if (row_ok) {
-#pragma unroll
-                for (int e8 = 0; e8 < 4; ++e8) {
-                    uint4 pk;
-                    pk.x = pack_bf16(ov[e8 * 8 + 0] * inv_l, ov[e8 * 8 + 1] * inv_l);
-                    pk.y = pack_bf16(ov[e8 * 8 + 2] * inv_l, ov[e8 * 8 + 3] * inv_l);
-                    pk.z = pack_bf16(ov[e8 * 8 + 4] * inv_l, ov[e8 * 8 + 5] * inv_l);
-                    pk.w = pack_bf16(ov[e8 * 8 + 6] * inv_l, ov[e8 * 8 + 7] * inv_l);
-                    *reinterpret_cast<uint4*>(orow + c * 32 + e8 * 8) = pk;
+                    for (int e8 = 0; e8 < 4; ++e8) {
+                        uint4 pk;
+                        pk.x = pack_bf16(ov[e8 * 8 + 0] * inv_l, ov[e8 * 8 + 1] * inv_l);
+                        pk.y = pack_bf16(ov[e8 * 8 + 2] * inv_l, ov[e8 * 8 + 3] * inv_l);
+                        pk.z = pack_bf16(ov[e8 * 8 + 4] * inv_l, ov[e8 * 8 + 5] * inv_l);
+                        pk.w = pack_bf16(ov[e8 * 8 + 6] * inv_l, ov[e8 * 8 + 7] * inv_l);
+                        *reinterpret_cast<uint4*>(orow + c * 32 + e8 * 8) = pk;
+                    }
                 }
             }
+            if (row_ok)
+                prm.lse[(size_t)h * prm.T + tok] = (m_ref + __log2f(l_run)) * 0.69314718055994531f;
         }
-        if (row_ok)
-            prm.lse[(size_t)h * prm.T + t] = (m_run + __log2f(l_run)) * 0.69314718055994531f;
     }
-    if (!ok && tid == 0) {
-        // a wait gave up: let this CTA's own TMA copies land (bounded) before exit
-        if (!q_waited) mbar_wait(bar_q, 0, 5);
-        for (int st = 0; st < 2; ++st)
-            while (kv_waited[st] < kv_issued[st] && mbar_wait(&bar_kv[st], kv_waited[st] & 1, 5))
-                ++kv_waited[st];
-    }
+
     tc_fence_before();
     __syncthreads();
-    if (warp == 0) tmem_dealloc(tmem, 256);
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
 }
 
 }  // namespace lf
