@@ -484,22 +484,34 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 tc_fence_after();
                 const int qh = q0 + hf * 64;
                 const bool live = lane_used && qh < len && (hf ? e.w1 : e.w0) != 0.f;
+                // copy the half's dQ^T to registers and hand its TMEM columns back to
+                // the MMA issuer at once; the reductions follow off its critical path
+                float v[64];
                 if (live) {
                     const uint32_t t_q = tmem + 256 + hf * 128 + lane_off;
-                    // head-major accumulator: the half's 64 query rows are contiguous
-                    float* dst = prm.dq_acc + ((size_t)e.h * prm.T + seg0 + qh) * D + dd;
-                    const int nvalid = min(64, len - qh);
+                    uint32_t a[16], b[16];
 #pragma unroll
-                    for (int c = 0; c < 2; ++c) {
-                        float v[32];
-                        tmem_ld32(t_q + c * 32, v);
+                    for (int c = 0; c < 4; c += 2) {
+                        tmem_ld16_nowait(t_q + c * 16, a);
+                        tmem_ld16_nowait(t_q + (c + 1) * 16, b);
+                        tmem_wait_ld_regs(a, b);
 #pragma unroll
-                        for (int q = 0; q < 32; ++q)
-                            if (c * 32 + q < nvalid) atomicAdd(dst + (c * 32 + q) * D, v[q]);
+                        for (int e2 = 0; e2 < 16; ++e2) {
+                            v[c * 16 + e2] = __uint_as_float(a[e2]);
+                            v[(c + 1) * 16 + e2] = __uint_as_float(b[e2]);
+                        }
                     }
                 }
                 tc_fence_before();
                 mbar_arrive(&bar_dq_free[hf]);
+                if (live) {
+                    // head-major accumulator: the half's 64 query rows are contiguous
+                    float* dst = prm.dq_acc + ((size_t)e.h * prm.T + seg0 + qh) * D + dd;
+                    const int nvalid = min(64, len - qh);
+#pragma unroll
+                    for (int q = 0; q < 64; ++q)
+                        if (q < nvalid) atomicAdd(dst + q * D, v[q]);
+                }
             }
             if (!ok) break;
             ++n;
