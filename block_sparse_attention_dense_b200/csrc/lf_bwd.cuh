@@ -184,7 +184,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_init(&bar_qdo_full[i], 1);
             mbar_init(&bar_qdo_empty[i], 1);
             mbar_init(&bar_s_full[i], 1);
-            mbar_init(&bar_p_ready[i], 128);
+            mbar_init(&bar_p_ready[i], 256);
             mbar_init(&bar_dq_full[i], 1);
             mbar_init(&bar_dq_free[i], 128);
         }
@@ -349,20 +349,18 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         __syncwarp();
     } else if ((warp >= 4 && warp < 8) || warp >= 12) {
-        // ============ element-wise, one warpgroup per half (thread = KV row) ============
-        const int hf = warp >= 12 ? 1 : 0;                // the half this warpgroup owns
-        const int bar_id = hf ? 3 : 1;
+        // ===== element-wise: both warpgroups on each half, 32 columns each (thread = KV row) =====
+        const int wg = warp >= 12 ? 1 : 0;                // columns [32 wg, 32 wg + 32) of a half
+        const int hf_epi = wg;                            // epilogue: 0 -> dV, 1 -> dK
         const int r = (warp & 3) * 32 + lane;             // TMEM lane / KV row
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const int kv_local = jt * 128 + r;
         const bool kv_valid = kv_local < len;
-        const uint32_t t_s = tmem + 256 + hf * 128 + lane_off, t_dp = t_s + 64;
-        const uint32_t dsa = s_base + L::kDS + hf * L::kHalfDS;
         int n = 0;
         bool more = any, failed = false;
         for (;;) {
-            // uniform decision of the warpgroup; also: all are done with the old vectors
-            if (named_bar_or(bar_id, 128, !more || failed)) break;
+            // uniform decision of both warpgroups; also: all are done with the old vectors
+            if (named_bar_or(1, 256, !more || failed)) break;
             const bool got_e = mbar_wait_or_abort(&bar_entry[n & 3], (n >> 2) & 1, 41, abort_flag);
             const PairEntry e = ring[n & 3];
             if (!got_e || e.h < 0) {
@@ -372,7 +370,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
             const int qt = e.tile, q0 = qt * 128;
             if (r < 64) {
-                const int col = hf * 64 + r;
+                // this warpgroup's 64 columns: [32 wg, 32 wg + 32) of each half
+                const int col = (r >> 5) * 64 + wg * 32 + (r & 31);
                 const int q_local = q0 + col;
                 float l2 = INFINITY, dd = 0.f;    // exp2(S - inf) = 0: columns past the segment vanish
                 if (q_local < len) {
@@ -383,65 +382,65 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 lse2_s[col] = l2;
                 dvec_s[col] = dd;
             }
-            named_bar_sync(bar_id, 128);
+            named_bar_sync(2, 256);
             const bool diag = prm.causal && qt == jt;
-            const float w = kv_valid ? (hf ? e.w1 : e.w0) : 0.f;
-            const bool got = mbar_wait_or_abort(&bar_s_full[hf], n & 1, 38, abort_flag);
-            if (!__all_sync(0xffffffffu, got)) { failed = true; continue; }
-            tc_fence_after();
-            // 16-column chunks; the next chunk's TMEM loads overlap this chunk's math
-            auto chunk = [&](int c, const uint32_t (&sr)[16], const uint32_t (&dr)[16]) {
-                uint32_t pk[8], dk_[8];
-#pragma unroll
-                for (int e4 = 0; e4 < 4; ++e4) {
-                    const int col0 = hf * 64 + c * 16 + 4 * e4;
-                    const float4 l4 = *reinterpret_cast<const float4*>(lse2_s + col0);
-                    const float4 d4 = *reinterpret_cast<const float4*>(dvec_s + col0);
-                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-                    const float dv_[4] = {d4.x, d4.y, d4.z, d4.w};
-                    float pw[4], dsw[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) {
-                        float p = fast_exp2(fmaf(__uint_as_float(sr[4 * e4 + u]), prm.scale_log2, -lv[u]));
-                        if (diag && kv_local > q0 + col0 + u) p = 0.f;
-                        pw[u] = p * w;
-                        dsw[u] = pw[u] * (__uint_as_float(dr[4 * e4 + u]) - dv_[u]);
-                    }
-                    pk[2 * e4] = pack_bf16(pw[0], pw[1]);
-                    pk[2 * e4 + 1] = pack_bf16(pw[2], pw[3]);
-                    dk_[2 * e4] = pack_bf16(dsw[0], dsw[1]);
-                    dk_[2 * e4 + 1] = pack_bf16(dsw[2], dsw[3]);
+            for (int hf = 0; hf < 2; ++hf) {
+                const float w = kv_valid ? (hf ? e.w1 : e.w0) : 0.f;
+                const uint32_t t_s = tmem + 256 + hf * 128 + lane_off, t_dp = t_s + 64;
+                const uint32_t dsa = s_base + L::kDS + hf * L::kHalfDS;
+                const bool got = mbar_wait_or_abort(&bar_s_full[hf], n & 1, 38, abort_flag);
+                const bool ok = __all_sync(0xffffffffu, got);
+                // this warpgroup's two 16-column chunks of S^T and dP^T
+                uint32_t sa[16], da[16], sb[16], db[16];
+                if (ok) {
+                    tc_fence_after();
+                    tmem_ld16_nowait(t_s + (2 * wg) * 16, sa);
+                    tmem_ld16_nowait(t_dp + (2 * wg) * 16, da);
+                    tmem_ld16_nowait(t_s + (2 * wg + 1) * 16, sb);
+                    tmem_ld16_nowait(t_dp + (2 * wg + 1) * 16, db);
+                    tmem_wait_ld_regs(sa, da);
+                    tmem_wait_ld_regs(sb, db);
                 }
-                // P^T over S^T (packed columns [8c, 8c+8)), dS^T over dP^T: columns
-                // whose fp32 values were read by earlier chunks
-                tmem_st8(t_s + c * 8, pk);
-                tmem_st8(t_dp + c * 8, dk_);
-                // dS^T into shared memory (one 64-column panel, SW128)
-                st_shared_v4(dsa + sw128_chunk_offset(r, 2 * c), dk_[0], dk_[1], dk_[2], dk_[3]);
-                st_shared_v4(dsa + sw128_chunk_offset(r, 2 * c + 1), dk_[4], dk_[5], dk_[6], dk_[7]);
-            };
-            uint32_t sa[16], da[16], sb[16], db[16];
-            tmem_ld16_nowait(t_s, sa);
-            tmem_ld16_nowait(t_dp, da);
-            tmem_wait_ld_regs(sa, da);
-            tmem_ld16_nowait(t_s + 16, sb);
-            tmem_ld16_nowait(t_dp + 16, db);
-            chunk(0, sa, da);
-            tmem_wait_ld_regs(sb, db);
-            tmem_ld16_nowait(t_s + 32, sa);
-            tmem_ld16_nowait(t_dp + 32, da);
-            chunk(1, sb, db);
-            tmem_wait_ld_regs(sa, da);
-            tmem_ld16_nowait(t_s + 48, sb);
-            tmem_ld16_nowait(t_dp + 48, db);
-            chunk(2, sa, da);
-            tmem_wait_ld_regs(sb, db);
-            chunk(3, sb, db);
-            tmem_wait_st();
-            fence_proxy_async_smem();
-            tc_fence_before();
-            mbar_arrive(&bar_p_ready[hf]);
-            ++n;
+                // every fp32 column of the half is in registers before P^T/dS^T are
+                // written over them (the packed columns of one warpgroup overlap the
+                // fp32 columns of the other)
+                named_bar_sync(3, 256);
+                if (!ok) { failed = true; continue; }
+                auto chunk = [&](int c, const uint32_t (&sr)[16], const uint32_t (&dr)[16]) {
+                    uint32_t pk[8], dk_[8];
+#pragma unroll
+                    for (int e4 = 0; e4 < 4; ++e4) {
+                        const int col0 = hf * 64 + c * 16 + 4 * e4;
+                        const float4 l4 = *reinterpret_cast<const float4*>(lse2_s + col0);
+                        const float4 d4 = *reinterpret_cast<const float4*>(dvec_s + col0);
+                        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+                        const float dv_[4] = {d4.x, d4.y, d4.z, d4.w};
+                        float pw[4], dsw[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            float p = fast_exp2(fmaf(__uint_as_float(sr[4 * e4 + u]), prm.scale_log2, -lv[u]));
+                            if (diag && kv_local > q0 + col0 + u) p = 0.f;
+                            pw[u] = p * w;
+                            dsw[u] = pw[u] * (__uint_as_float(dr[4 * e4 + u]) - dv_[u]);
+                        }
+                        pk[2 * e4] = pack_bf16(pw[0], pw[1]);
+                        pk[2 * e4 + 1] = pack_bf16(pw[2], pw[3]);
+                        dk_[2 * e4] = pack_bf16(dsw[0], dsw[1]);
+                        dk_[2 * e4 + 1] = pack_bf16(dsw[2], dsw[3]);
+                    }
+                    tmem_st8(t_s + c * 8, pk);     // P^T, packed columns [8c, 8c+8)
+                    tmem_st8(t_dp + c * 8, dk_);   // dS^T
+                    st_shared_v4(dsa + sw128_chunk_offset(r, 2 * c), dk_[0], dk_[1], dk_[2], dk_[3]);
+                    st_shared_v4(dsa + sw128_chunk_offset(r, 2 * c + 1), dk_[4], dk_[5], dk_[6], dk_[7]);
+                };
+                chunk(2 * wg, sa, da);
+                chunk(2 * wg + 1, sb, db);
+                tmem_wait_st();
+                fence_proxy_async_smem();
+                tc_fence_before();
+                mbar_arrive(&bar_p_ready[hf]);
+            }
+            if (!failed) ++n;
         }
         // ---- epilogue: warpgroup 0 adds dV, warpgroup 1 adds dK (unscaled) into the
         // fp32 accumulators of the KV head (the GQA sum over query heads) ----
@@ -450,8 +449,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         have = __all_sync(0xffffffffu, have);
         if (have) {
             tc_fence_after();
-            float* dst = (hf ? prm.dk_acc : prm.dv_acc) + ((size_t)(kv_row0 + r) * prm.hkv + g) * D;
-            const uint32_t t_acc = (hf ? t_dk : t_dv) + lane_off;
+            float* dst = (hf_epi ? prm.dk_acc : prm.dv_acc) + ((size_t)(kv_row0 + r) * prm.hkv + g) * D;
+            const uint32_t t_acc = (hf_epi ? t_dk : t_dv) + lane_off;
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
                 float v[32];
