@@ -151,6 +151,13 @@ def lf_attn_bwd(desc, q, k, v, o, lse, dout, D, block_weight, kept_idx, kept_cnt
                                _stream(stream)), "lf_attn_bwd")
 
 
+def lf_watchdog_selftest(limit_log2=24, stream=None):
+    L = _load()
+    L.lf_watchdog_selftest.argtypes = [ctypes.c_uint32, ctypes.c_void_p]
+    L.lf_watchdog_selftest.restype = ctypes.c_int
+    _check(L.lf_watchdog_selftest(int(limit_log2), _stream(stream)), "lf_watchdog_selftest")
+
+
 def lf_check_device_error(stream=None):
     _check(_load().lf_check_device_error(_stream(stream)), "lf_check_device_error")
 

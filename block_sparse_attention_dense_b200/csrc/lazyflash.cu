@@ -195,6 +195,22 @@ lf_status launch_bwd(const lf_attn_desc* d, const void* q, const void* k, const 
 
 }  // namespace
 
+namespace lf {
+// Failure-detection self-test: one thread waits, with the kernels' bounded wait,
+// on a barrier phase that nothing completes.  The wait gives up after `limit`
+// cycles and records a timeout in the device flag; nothing faults or traps.
+__global__ void watchdog_selftest_kernel(long long limit) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        fence_barrier_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, 99, limit);
+    __syncthreads();
+}
+}  // namespace lf
+
 // Scratch of lf_attn_bwd_static_ws: one array per device, loaded with the
 // library and kept until the process exits.  Host code must not use this name
 // as a device address (it names a host-side stand-in); the device address comes
@@ -370,6 +386,13 @@ lf_status lf_attn_bwd_static_ws(const lf_attn_desc* desc, const void* q, const v
                                             kept_cnt, dq, dk, dv, ws, s)
                           : launch_bwd<64>(desc, q, k, v, lse, dout, Dv, block_weight, kept_idx,
                                            kept_cnt, dq, dk, dv, ws, s);
+}
+
+lf_status lf_watchdog_selftest(uint32_t limit_log2, lf_stream_t stream) {
+    if (limit_log2 < 10 || limit_log2 > 31) return LF_ERR_INVALID_ARG;
+    lf::watchdog_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+        1ll << limit_log2);
+    return launch_status();
 }
 
 lf_status lf_check_device_error(lf_stream_t stream) {

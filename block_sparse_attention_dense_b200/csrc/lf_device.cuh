@@ -85,12 +85,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Waits until the phase with the given parity has completed.  Returns false
-// (and records `site`) if that takes longer than kWaitLimitCycles.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int site) {
+// (and records `site`) if that takes longer than `limit` SM cycles.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int site,
+                                          long long limit = kWaitLimitCycles) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (!mbar_try_wait(bar, parity)) {
-        if (clock64() - t0 > kWaitLimitCycles) {
+        if (clock64() - t0 > limit) {
             report_timeout(site);
             return false;
         }

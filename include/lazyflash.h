@@ -163,6 +163,14 @@ lf_status lf_attn_bwd_static_ws(const lf_attn_desc* desc, const void* q, const v
                                 const int32_t* kept_idx, const int32_t* kept_cnt, void* dq,
                                 void* dk, void* dv, lf_stream_t stream);
 
+/* Failure-detection self-test (no counterpart in the article): launches one
+ * CTA whose bounded barrier wait, the one every kernel uses, waits for a phase
+ * that nothing completes and gives up after 2^limit_log2 SM cycles (10..31),
+ * recording a timeout in the device flag.  Nothing faults or traps: after
+ * lf_check_device_error returns LF_ERR_TIMEOUT the context stays usable.
+ * Returns LF_ERR_INVALID_ARG for a limit outside 10..31. */
+lf_status lf_watchdog_selftest(uint32_t limit_log2, lf_stream_t stream);
+
 /* Waits for `stream`, then reads and clears the device watchdog flag.
  * LF_ERR_TIMEOUT if a kernel gave up a bounded wait since the last check,
  * LF_ERR_CUDA if the stream reported an error, else LF_OK. */
