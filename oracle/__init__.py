@@ -65,6 +65,14 @@ def lib():
                                      ctypes.POINTER(ctypes.c_uint8), i32p, i32p]
             L.lfo_attn_bwd.argtypes = [c_int, i32p, c_int, c_int, c_int, c_int, c_dbl, c_int,
                                        c_int, c_int, dp, dp, dp, dp, dp, dp, dp, dp]
+            L.lfo_select_rule.argtypes = [c_int, c_int, i32p, c_int, c_int, dp, c_dbl,
+                                          ctypes.c_uint64, ctypes.c_uint64, dp, dp,
+                                          ctypes.POINTER(ctypes.c_float),
+                                          ctypes.POINTER(ctypes.c_uint8), i32p, i32p]
+            L.lfo_tau_fixed_fraction.argtypes = [dp, c_int, c_dbl]
+            L.lfo_tau_fixed_fraction.restype = c_dbl
+            L.lfo_expected_kept.argtypes = [dp, c_int, c_dbl, dp]
+            L.lfo_expected_kept.restype = c_dbl
             L.lfo_attn_fwd_rows.argtypes = [c_int, i32p, c_int, c_int, c_int, c_int, c_dbl, c_int,
                                             dp, dp, dp, c_int, i32p, i32p, dp, dp]
             L.lfo_attn_bwd_rows.argtypes = [c_int, i32p, c_int, c_int, c_int, c_int, c_dbl, c_int,
@@ -258,3 +266,34 @@ def attn_bwd_rows(cu_seqlens, q, k, v, dout, scale: float, block: int, wblk, qro
                                    len(kvrows), _p(kvrows, ip), _p(kvheads, ip), _p(dk, dp),
                                    _p(dv, dp)), "attn_bwd_rows")
     return dq, dk, dv
+
+
+RULE_BUDGET, RULE_FIXED_FRACTION, RULE_TOPK = 0, 1, 2
+
+
+def select_rule(rule: int, norms, nb, param: float, seed: int, step: int) -> dict:
+    """Selection by rule 0 (budget delta = param), 1 (fixed fraction f = param)
+    or 2 (top-k with k = ceil(param * n)); same outputs as select()."""
+    m = _f64(norms)
+    nseq, hq, nbmax = m.shape
+    nb = _i32(nb)
+    out = {
+        "tau": np.zeros((nseq, hq), dtype=np.float64),
+        "p": np.zeros((nseq, hq, nbmax), dtype=np.float64),
+        "w": np.zeros((nseq, hq, nbmax), dtype=np.float32),
+        "keep": np.zeros((nseq, hq, nbmax), dtype=np.uint8),
+        "kept_idx": np.zeros((nseq, hq, nbmax), dtype=np.int32),
+        "kept_cnt": np.zeros((nseq, hq), dtype=np.int32),
+    }
+    dp = ctypes.c_double
+    _check(lib().lfo_select_rule(int(rule), nseq, _p(nb, ctypes.c_int32), hq, nbmax, _p(m, dp),
+                                 float(param), int(seed) & (2**64 - 1), int(step) & (2**64 - 1),
+                                 _p(out["tau"], dp), _p(out["p"], dp), _p(out["w"], ctypes.c_float),
+                                 _p(out["keep"], ctypes.c_uint8), _p(out["kept_idx"], ctypes.c_int32),
+                                 _p(out["kept_cnt"], ctypes.c_int32)), "select_rule")
+    return out
+
+
+def tau_fixed_fraction(m, f: float) -> float:
+    m = _f64(m)
+    return float(lib().lfo_tau_fixed_fraction(_p(m, ctypes.c_double), len(m), f))

@@ -544,3 +544,112 @@ int lfo_attn_bwd_rows(int nseq, const int32_t* cu, int T, int hq, int hkv, int d
     free(done); free(members);
     return LFO_OK;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Alternative selection rules compared by the article at equal backward     */
+/* time (section "Le choix des blocs pèse plus que la quantité sautée"):      */
+/*  rule 1, fixed fraction f: the same proportional draw and 1/p weights, but */
+/*    tau is the largest threshold whose expected kept count                  */
+/*    sum_b min(1, m_b/tau) is at least f*n (a fraction fixed for the whole   */
+/*    run instead of the adaptive mass budget);                               */
+/*  rule 2, top-k: the k = ceil(f*n) largest norms (ties: lower index), kept  */
+/*    deterministically with weight 1 (the same blocks at every step).        */
+/* tau reports the threshold (rule 1) or the k-th largest norm (rule 2).      */
+/* ------------------------------------------------------------------------ */
+double lfo_expected_kept(const double* m, int n, double tau, double* scratch)
+{
+    for (int b = 0; b < n; ++b) scratch[b] = (m[b] >= tau) ? 1.0 : m[b] / tau;
+    return lfo_pinned_sum(scratch, n);
+}
+
+double lfo_tau_fixed_fraction(const double* m, int n, double f)
+{
+    double* scratch = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
+    double M = lfo_pinned_sum(m, n);
+    double tau = 0.0;
+    if (n > 0 && M > 0.0 && f < 1.0) {
+        double target = f * (double)n;
+        double lo = 0.0, hi = M / target;
+        for (int it = 0; it < 64; ++it) {
+            double mid = 0.5 * (lo + hi);
+            double g = lfo_expected_kept(m, n, mid, scratch);
+            if (g >= target) lo = mid; else hi = mid;
+        }
+        tau = lo;
+    }
+    free(scratch);
+    return tau;
+}
+
+static int topk_count(int n, double f)
+{
+    double kd = ceil(f * (double)n);
+    int k = (int)kd;
+    if (k > n) k = n;
+    if (k < 0) k = 0;
+    return k;
+}
+
+int lfo_select_rule(int rule, int nseq, const int32_t* nb, int hq, int nbmax, const double* norms,
+                    double param, uint64_t seed, uint64_t step,
+                    double* tau, double* p, float* w, uint8_t* keep,
+                    int32_t* kept_idx, int32_t* kept_cnt)
+{
+    if (rule == 0)
+        return lfo_select(nseq, nb, hq, nbmax, norms, param, seed, step, tau, p, w, keep,
+                          kept_idx, kept_cnt);
+    if (rule != 1 && rule != 2) return LFO_EINVAL;
+    if (nseq < 1 || hq < 1 || nbmax < 1 || !(param > 0.0 && param <= 1.0)) return LFO_EINVAL;
+    for (int s = 0; s < nseq; ++s) if (nb[s] < 0 || nb[s] > nbmax) return LFO_EINVAL;
+    #pragma omp parallel for collapse(2)
+    for (int s = 0; s < nseq; ++s)
+        for (int h = 0; h < hq; ++h) {
+            size_t base = ((size_t)s * hq + h) * nbmax;
+            const double* m = norms + base;
+            int n = nb[s];
+            int cnt = 0;
+            if (rule == 1) {
+                double t = lfo_tau_fixed_fraction(m, n, param);
+                tau[(size_t)s * hq + h] = t;
+                for (int i = 0; i < nbmax; ++i) {
+                    double pi = 0.0;
+                    int kb = 0;
+                    float wi = 0.0f;
+                    if (i < n) {
+                        if (t == 0.0) pi = 1.0;
+                        else { pi = m[i] / t; if (pi > 1.0) pi = 1.0; }
+                        if (pi >= 1.0) kb = 1;
+                        else kb = ((double)lfo_block_u24(seed, step, s, h, i) < pi * 16777216.0);
+                        if (kb) wi = (float)(1.0 / pi);
+                    }
+                    p[base + i] = pi;
+                    keep[base + i] = (uint8_t)kb;
+                    w[base + i] = wi;
+                    kept_idx[base + i] = -1;
+                    if (kb) kept_idx[base + cnt++] = i;
+                }
+            } else {
+                int k = topk_count(n, param);
+                double kth = 0.0;
+                for (int i = 0; i < nbmax; ++i) {
+                    int kb = 0;
+                    if (i < n) {
+                        /* rank: blocks with a larger norm, or an equal norm and lower index */
+                        int rank = 0;
+                        for (int j = 0; j < n; ++j)
+                            if (m[j] > m[i] || (m[j] == m[i] && j < i)) ++rank;
+                        kb = rank < k;
+                        if (rank == k - 1) kth = m[i];
+                    }
+                    p[base + i] = kb ? 1.0 : 0.0;
+                    keep[base + i] = (uint8_t)kb;
+                    w[base + i] = kb ? 1.0f : 0.0f;
+                    kept_idx[base + i] = -1;
+                    if (kb) kept_idx[base + cnt++] = i;
+                }
+                tau[(size_t)s * hq + h] = kth;
+            }
+            kept_cnt[(size_t)s * hq + h] = cnt;
+        }
+    return LFO_OK;
+}

@@ -215,3 +215,90 @@ def test_sampled_gradient_unbiased_tiny():
     assert np.all(np.abs(z) < 4.0), z
     # and the empirical variance agrees with the exact one
     np.testing.assert_allclose(est.var(axis=0), var, rtol=0.15)
+
+
+# ---------------------------------------------------------------------------
+# Alternative rules (article section "Le choix des blocs pèse plus que la
+# quantité sautée"): fixed fraction and top-k.
+# ---------------------------------------------------------------------------
+def _tau_fixed_closed_form(m, f):
+    """On (m_(j+1), m_(j)] of the descending order the expected kept count is
+    j + S/tau, S the sum of the smaller norms: solve j + S/tau = f n on the
+    piece where the count crosses f n."""
+    m = np.sort(np.asarray(m, dtype=np.float64))[::-1]
+    n = len(m)
+    target = f * n
+    for j in range(0, n):
+        S = math.fsum(m[j:])
+        hi = m[j - 1] if j > 0 else math.inf     # tau <= hi keeps the j largest outright
+        lo = m[j]
+        if target - j <= 0:
+            continue
+        t = S / (target - j)
+        if lo <= t <= hi:
+            return t
+    raise AssertionError("no crossing")
+
+
+@pytest.mark.parametrize("seed", range(10))
+@pytest.mark.parametrize("f", [0.05, 0.2, 0.5, 0.9])
+def test_fixed_fraction_tau_matches_closed_form(seed, f):
+    rng = np.random.default_rng(200 + seed)
+    m = rng.lognormal(0.0, 2.0, size=int(rng.integers(2, 400)))
+    t = oracle.tau_fixed_fraction(m, f)
+    ref = _tau_fixed_closed_form(m, f)
+    assert abs(t - ref) <= 1e-12 * ref, (t, ref)
+    # expected kept count hits the target; a slightly larger tau falls short
+    p = np.minimum(1.0, m / t)
+    assert abs(math.fsum(p) - f * len(m)) <= 1e-9 * f * len(m)
+    assert math.fsum(np.minimum(1.0, m / (t * (1 + 1e-9)))) < f * len(m)
+
+
+def test_fixed_fraction_selection_outputs():
+    nb = np.array([100, 37], dtype=np.int32)
+    m = synthetic.random_norms(2, 3, 100, nb, 1.5, seed=8)
+    r = oracle.select_rule(oracle.RULE_FIXED_FRACTION, m, nb, 0.25, seed=4, step=6)
+    for s in range(2):
+        for h in range(3):
+            n = int(nb[s])
+            t = r["tau"][s, h]
+            p = np.minimum(1.0, m[s, h, :n].astype(np.float64) / t)
+            np.testing.assert_array_equal(r["p"][s, h, :n], p)
+            for i in range(n):
+                u = oracle.block_u24(4, 6, s, h, i)
+                assert bool(r["keep"][s, h, i]) == (p[i] >= 1.0 or u < p[i] * 2.0 ** 24)
+            kept = np.nonzero(r["keep"][s, h, :n])[0]
+            np.testing.assert_array_equal(r["kept_idx"][s, h, :len(kept)], kept)
+            np.testing.assert_array_equal(r["w"][s, h, kept], (1.0 / p[kept]).astype(np.float32))
+
+
+@pytest.mark.parametrize("f", [0.01, 0.1, 0.33, 1.0])
+def test_topk_matches_library_sort(f):
+    nb = np.array([256, 57], dtype=np.int32)
+    m = synthetic.random_norms(2, 4, 256, nb, 2.0, seed=9)
+    m[1, 2, 10:20] = m[1, 2, 5]                  # ties: the lower index wins
+    r = oracle.select_rule(oracle.RULE_TOPK, m, nb, f, seed=0, step=0)
+    for s in range(2):
+        for h in range(4):
+            n = int(nb[s])
+            k = min(n, math.ceil(f * n))
+            order = np.lexsort((np.arange(n), -m[s, h, :n].astype(np.float64)))
+            want = np.sort(order[:k])
+            kept = np.nonzero(r["keep"][s, h, :n])[0]
+            np.testing.assert_array_equal(kept, want)
+            assert r["kept_cnt"][s, h] == k
+            assert np.all(r["w"][s, h, kept] == 1.0)
+            if k:
+                assert r["tau"][s, h] == m[s, h, order[k - 1]]
+    # top-k is the same at every step (deterministic)
+    r2 = oracle.select_rule(oracle.RULE_TOPK, m, nb, f, seed=5, step=77)
+    np.testing.assert_array_equal(r["keep"], r2["keep"])
+
+
+def test_rule_zero_is_the_budget_rule():
+    nb = np.array([64], dtype=np.int32)
+    m = synthetic.random_norms(1, 2, 64, nb, 1.5, seed=1)
+    a = oracle.select_rule(oracle.RULE_BUDGET, m, nb, 0.1, 3, 4)
+    b = oracle.select(m, nb, 0.1, 3, 4)
+    for k_ in a:
+        np.testing.assert_array_equal(a[k_], b[k_])
