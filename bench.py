@@ -182,7 +182,8 @@ def config_of(w, args):
     return {"workload": w.name, "seqlens": list(w.seqlens) if w.nseq <= 16 else "%d segments" % w.nseq,
             "total_tokens": w.total_tokens, "hq": w.hq, "hkv": w.hkv, "d": w.d, "block": w.block,
             "causal": w.causal, "delta": w.delta, "dO_block_scale": "LogNormal(0,%g)" % w.sigma,
-            "seed": 0, "step": 0,
+            "seed": 0, "step": 0, "rule": args.rule if hasattr(args, "rule") else "budget",
+            "rule_param": getattr(args, "rule_param", None),
             "l2": "no flush: every input tensor (>= 64 MiB x4 heads) exceeds L2 per step",
             "parallelism": "replicas" if args.gpus > 1 else "single"}
 
@@ -198,6 +199,12 @@ def main():
     ap.add_argument("--impl", default="lazyflash", choices=["lazyflash", "reference"])
     ap.add_argument("--workload", default="headline", choices=sorted(synthetic.WORKLOADS))
     ap.add_argument("--delta", type=float, default=None)
+    ap.add_argument("--rule", default="budget", choices=["budget", "fixed", "topk"],
+                    help="selection rule (budget = LazyFlash; fixed fraction and top-k are the "
+                         "article's comparison rules); --rule-param is f for the latter two")
+    ap.add_argument("--rule-param", type=float, default=None)
+    ap.add_argument("--seqlen", type=int, default=None, help="override the workload's length "
+                    "(single-segment workloads)")
     ap.add_argument("--cpu-prefix", type=int, default=2048,
                     help="tokens of the oracle sample timed for cpu_baseline")
     ap.add_argument("--ref-prefix", type=int, default=1024,
@@ -208,6 +215,14 @@ def main():
     w = synthetic.WORKLOADS[args.workload]
     if args.delta is not None:
         w = w.with_(delta=args.delta)
+    if args.seqlen is not None:
+        if w.nseq != 1:
+            raise SystemExit("--seqlen applies to single-segment workloads")
+        w = w.with_(seqlens=(args.seqlen,))
+    rule_id = {"budget": 0, "fixed": 1, "topk": 2}[args.rule]
+    rule_param = w.delta if rule_id == 0 else args.rule_param
+    if rule_id != 0 and rule_param is None:
+        raise SystemExit("--rule fixed/topk needs --rule-param f")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -239,10 +254,13 @@ def main():
                         w.block)
     bufs = lf.Buffers(desc, device=dev)
 
+    def select():
+        lf.lf_block_select_rule(desc, d_in["dout"], bufs.o, rule_id, rule_param, 0, 0, 0, bufs.norm,
+                                bufs.D, bufs.tau, bufs.w, bufs.keep, bufs.kept_idx, bufs.kept_cnt)
+
     def step():
         lf.lf_attn_fwd(desc, d_in["q"], d_in["k"], d_in["v"], bufs.o, bufs.lse)
-        lf.lf_block_select(desc, d_in["dout"], bufs.o, w.delta, 0, 0, 0, bufs.norm, bufs.D,
-                           bufs.tau, bufs.w, bufs.keep, bufs.kept_idx, bufs.kept_cnt)
+        select()
         lf.lf_attn_bwd(desc, d_in["q"], d_in["k"], d_in["v"], bufs.o, bufs.lse, d_in["dout"],
                        bufs.D, bufs.w, bufs.kept_idx, bufs.kept_cnt, bufs.dq, bufs.dk, bufs.dv,
                        bufs.ws)
@@ -269,8 +287,7 @@ def main():
         e[0].record(stream)
         lf.lf_attn_fwd(desc, d_in["q"], d_in["k"], d_in["v"], bufs.o, bufs.lse)
         e[1].record(stream)
-        lf.lf_block_select(desc, d_in["dout"], bufs.o, w.delta, 0, 0, 0, bufs.norm, bufs.D,
-                           bufs.tau, bufs.w, bufs.keep, bufs.kept_idx, bufs.kept_cnt)
+        select()
         e[2].record(stream)
         lf.lf_attn_bwd(desc, d_in["q"], d_in["k"], d_in["v"], bufs.o, bufs.lse, d_in["dout"],
                        bufs.D, bufs.w, bufs.kept_idx, bufs.kept_cnt, bufs.dq, bufs.dk, bufs.dv,

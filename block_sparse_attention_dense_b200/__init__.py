@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(_PKG, "liblazyflash.so")
 LF_OK, LF_ERR_INVALID_ARG, LF_ERR_UNSUPPORTED, LF_ERR_WORKSPACE, LF_ERR_CUDA, LF_ERR_TIMEOUT = range(6)
 LF_WS_FWD, LF_WS_SELECT, LF_WS_BWD = 0, 1, 2
 LF_SELECT_NORMS_GIVEN = 0x1
+LF_RULE_BUDGET, LF_RULE_FIXED_FRACTION, LF_RULE_TOPK = 0, 1, 2
 
 EXPORTED = ("lf_workspace_size", "lf_attn_fwd", "lf_block_select", "lf_attn_bwd",
             "lf_check_device_error", "lf_status_string")
@@ -140,6 +141,21 @@ def lf_block_select(desc, dout, o, delta, seed, step, flags, block_norm, D, tau,
                                    _ptr(keep), _ptr(kept_idx), _ptr(kept_cnt), _ptr(ws),
                                    0 if ws is None else ws.numel() * ws.element_size(),
                                    _stream(stream)), "lf_block_select")
+
+
+def lf_block_select_rule(desc, dout, o, rule, param, seed, step, flags, block_norm, D, tau,
+                         block_weight, keep, kept_idx, kept_cnt, ws=None, stream=None):
+    L = _load()
+    fn = L.lf_block_select_rule
+    fn.argtypes = [ctypes.POINTER(lf_attn_desc), ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int,
+                   ctypes.c_double, ctypes.c_uint64, ctypes.c_uint64, ctypes.c_uint32] + \
+        [ctypes.c_void_p] * 8 + [ctypes.c_size_t, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    _check(fn(ctypes.byref(desc), _ptr(dout), _ptr(o), int(rule), float(param),
+              int(seed) & (2**64 - 1), int(step) & (2**64 - 1), int(flags), _ptr(block_norm),
+              _ptr(D), _ptr(tau), _ptr(block_weight), _ptr(keep), _ptr(kept_idx), _ptr(kept_cnt),
+              _ptr(ws), 0 if ws is None else ws.numel() * ws.element_size(), _stream(stream)),
+           "lf_block_select_rule")
 
 
 def lf_attn_bwd(desc, q, k, v, o, lse, dout, D, block_weight, kept_idx, kept_cnt, dq, dk, dv,

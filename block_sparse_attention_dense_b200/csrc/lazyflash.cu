@@ -280,16 +280,20 @@ lf_status lf_attn_fwd(const lf_attn_desc* desc, const void* q, const void* k, co
                           : launch_fwd<64>(desc, q, k, v, o, lse, s);
 }
 
-lf_status lf_block_select(const lf_attn_desc* desc, const void* dout, const void* o, double delta,
-                          uint64_t seed, uint64_t step, uint32_t flags, float* block_norm,
-                          float* D, double* tau, float* block_weight, uint8_t* keep,
-                          int32_t* kept_idx, int32_t* kept_cnt, void* ws, size_t ws_bytes,
-                          lf_stream_t stream) {
-    (void)ws;
-    (void)ws_bytes;
+static lf_status block_select_impl(const lf_attn_desc* desc, const void* dout, const void* o,
+                                   int rule, double param, uint64_t seed, uint64_t step,
+                                   uint32_t flags, float* block_norm, float* D, double* tau,
+                                   float* block_weight, uint8_t* keep, int32_t* kept_idx,
+                                   int32_t* kept_cnt, lf_stream_t stream) {
     lf_status st = check_desc(desc);
     if (st != LF_OK) return st;
-    if (!(delta >= 0.0 && delta < 1.0)) return LF_ERR_INVALID_ARG;
+    if (rule == LF_RULE_BUDGET) {
+        if (!(param >= 0.0 && param < 1.0)) return LF_ERR_INVALID_ARG;
+    } else if (rule == LF_RULE_FIXED_FRACTION || rule == LF_RULE_TOPK) {
+        if (!(param > 0.0 && param <= 1.0)) return LF_ERR_INVALID_ARG;
+    } else {
+        return LF_ERR_INVALID_ARG;
+    }
     if (flags & ~LF_SELECT_NORMS_GIVEN) return LF_ERR_INVALID_ARG;
     if (!dout || !o || !block_norm || !D || !tau || !block_weight || !keep || !kept_idx ||
         !kept_cnt)
@@ -307,16 +311,39 @@ lf_status lf_block_select(const lf_attn_desc* desc, const void* dout, const void
                         : launch_norms<64>(desc, dout, o, block_norm, D, write_norms, s);
     if (st != LF_OK) return st;
     const size_t smem = (size_t)nbmax * sizeof(double);
+    auto kern = rule == LF_RULE_BUDGET ? lf::select_kernel<0>
+              : rule == LF_RULE_FIXED_FRACTION ? lf::select_kernel<1> : lf::select_kernel<2>;
     if (smem > 48 * 1024 &&
-        cudaFuncSetAttribute(lf::select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
+        cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess)
         return LF_ERR_CUDA;
     dim3 grid(desc->hq, desc->nseq);
-    lf::select_kernel<<<grid, 32, smem, s>>>(desc->cu_seqlens, desc->total_tokens,
-                                             desc->max_seqlen, desc->hq, desc->block_q, nbmax,
-                                             block_norm, delta, seed, step, tau, block_weight,
-                                             keep, kept_idx, kept_cnt);
+    kern<<<grid, 32, smem, s>>>(desc->cu_seqlens, desc->total_tokens, desc->max_seqlen, desc->hq,
+                                desc->block_q, nbmax, block_norm, param, seed, step, tau,
+                                block_weight, keep, kept_idx, kept_cnt);
     return launch_status();
+}
+
+lf_status lf_block_select(const lf_attn_desc* desc, const void* dout, const void* o, double delta,
+                          uint64_t seed, uint64_t step, uint32_t flags, float* block_norm,
+                          float* D, double* tau, float* block_weight, uint8_t* keep,
+                          int32_t* kept_idx, int32_t* kept_cnt, void* ws, size_t ws_bytes,
+                          lf_stream_t stream) {
+    (void)ws;
+    (void)ws_bytes;
+    return block_select_impl(desc, dout, o, LF_RULE_BUDGET, delta, seed, step, flags, block_norm,
+                             D, tau, block_weight, keep, kept_idx, kept_cnt, stream);
+}
+
+lf_status lf_block_select_rule(const lf_attn_desc* desc, const void* dout, const void* o,
+                               int rule, double param, uint64_t seed, uint64_t step,
+                               uint32_t flags, float* block_norm, float* D, double* tau,
+                               float* block_weight, uint8_t* keep, int32_t* kept_idx,
+                               int32_t* kept_cnt, void* ws, size_t ws_bytes, lf_stream_t stream) {
+    (void)ws;
+    (void)ws_bytes;
+    return block_select_impl(desc, dout, o, rule, param, seed, step, flags, block_norm, D, tau,
+                             block_weight, keep, kept_idx, kept_cnt, stream);
 }
 
 lf_status lf_attn_bwd(const lf_attn_desc* desc, const void* q, const void* k, const void* v,

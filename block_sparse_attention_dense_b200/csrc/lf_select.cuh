@@ -107,11 +107,17 @@ __device__ __forceinline__ double warp_butterfly_sum(double v) {
 
 // ---------------------------------------------------------------------------
 // 2. One warp per (segment, head).  Shared memory holds the head's norms as
-// fp64 (nbmax entries).
+// fp64 (nbmax entries).  RULE 0: the LazyFlash budget (param = delta): tau is
+// the largest threshold whose expected discarded mass sum (1 - p) m stays
+// within delta * sum m.  RULE 1: fixed fraction (param = f): tau is the
+// largest threshold whose expected kept count sum p reaches f * n.  Both draw
+// keep ~ Bernoulli(p = min(1, m/tau)) from Philox and weight kept blocks 1/p.
+// RULE 2: top-k (k = ceil(f * n)): the k largest norms, weight 1, no draw.
 // ---------------------------------------------------------------------------
+template <int RULE>
 __global__ void __launch_bounds__(32) select_kernel(
     const int32_t* __restrict__ cu_seqlens, int T, int max_seqlen, int hq, int block, int nbmax,
-    const float* __restrict__ norms, double delta, uint64_t seed, uint64_t step,
+    const float* __restrict__ norms, double param, uint64_t seed, uint64_t step,
     double* __restrict__ tau_out, float* __restrict__ w_out, uint8_t* __restrict__ keep_out,
     int32_t* __restrict__ kept_idx, int32_t* __restrict__ kept_cnt) {
     extern __shared__ double m_s[];
@@ -137,9 +143,10 @@ __global__ void __launch_bounds__(32) select_kernel(
     for (int off = 16; off > 0; off >>= 1) mx = fmax(mx, __shfl_xor_sync(0xffffffffu, mx, off));
 
     double tau = 0.0;
-    if (delta > 0.0 && total > 0.0) {
-        const double budget = __dmul_rn(delta, total);
-        double lo = 0.0, hi = __ddiv_rn(mx, __dsub_rn(1.0, delta));
+    int k_top = 0;
+    if (RULE == 0 && param > 0.0 && total > 0.0) {
+        const double budget = __dmul_rn(param, total);
+        double lo = 0.0, hi = __ddiv_rn(mx, __dsub_rn(1.0, param));
         for (int it = 0; it < 64; ++it) {
             const double mid = __dmul_rn(0.5, __dadd_rn(lo, hi));
             double f = 0.0;
@@ -152,8 +159,23 @@ __global__ void __launch_bounds__(32) select_kernel(
             if (f <= budget) lo = mid; else hi = mid;
         }
         tau = lo;
+    } else if (RULE == 1 && n > 0 && total > 0.0 && param < 1.0) {
+        const double target = __dmul_rn(param, static_cast<double>(n));
+        double lo = 0.0, hi = __ddiv_rn(total, target);
+        for (int it = 0; it < 64; ++it) {
+            const double mid = __dmul_rn(0.5, __dadd_rn(lo, hi));
+            double g = 0.0;
+            for (int i = lane; i < n; i += 32) {
+                const double m = m_s[i];
+                g = __dadd_rn(g, (m >= mid) ? 1.0 : __ddiv_rn(m, mid));
+            }
+            g = warp_butterfly_sum(g);
+            if (g >= target) lo = mid; else hi = mid;
+        }
+        tau = lo;
+    } else if (RULE == 2) {
+        k_top = min(n, static_cast<int>(ceil(__dmul_rn(param, static_cast<double>(n)))));
     }
-    if (lane == 0) tau_out[(size_t)s * hq + h] = tau;
 
     const uint2 key = make_uint2(static_cast<uint32_t>(seed), static_cast<uint32_t>(seed >> 32));
     int count = 0;
@@ -162,18 +184,31 @@ __global__ void __launch_bounds__(32) select_kernel(
         bool kept = false;
         float w = 0.f;
         if (i < n) {
-            double p = 1.0;
-            if (tau != 0.0) p = fmin(1.0, __ddiv_rn(m_s[i], tau));
-            if (p >= 1.0) {
-                kept = true;
+            if (RULE == 2) {
+                // rank = blocks with a larger norm, or an equal norm and a lower index
+                const double mi = m_s[i];
+                int rank = 0;
+                for (int j = 0; j < n; ++j) {
+                    const double mj = m_s[j];
+                    rank += (mj > mi || (mj == mi && j < i)) ? 1 : 0;
+                }
+                kept = rank < k_top;
+                if (rank == k_top - 1) tau = mi;
+                w = kept ? 1.f : 0.f;
             } else {
-                const uint4 r = philox4x32_10(
-                    make_uint4(static_cast<uint32_t>(i), static_cast<uint32_t>(h),
-                               static_cast<uint32_t>(s), static_cast<uint32_t>(step)),
-                    key);
-                kept = static_cast<double>(r.x >> 8) < __dmul_rn(p, 16777216.0);
+                double p = 1.0;
+                if (tau != 0.0) p = fmin(1.0, __ddiv_rn(m_s[i], tau));
+                if (p >= 1.0) {
+                    kept = true;
+                } else {
+                    const uint4 r = philox4x32_10(
+                        make_uint4(static_cast<uint32_t>(i), static_cast<uint32_t>(h),
+                                   static_cast<uint32_t>(s), static_cast<uint32_t>(step)),
+                        key);
+                    kept = static_cast<double>(r.x >> 8) < __dmul_rn(p, 16777216.0);
+                }
+                if (kept) w = __double2float_rn(__ddiv_rn(1.0, p));
             }
-            if (kept) w = __double2float_rn(__ddiv_rn(1.0, p));
         }
         if (i < nbmax) {
             keep_out[base + i] = kept ? 1 : 0;
@@ -184,7 +219,15 @@ __global__ void __launch_bounds__(32) select_kernel(
         count += __popc(ballot);
     }
     for (int i = count + lane; i < nbmax; i += 32) kept_idx[base + i] = -1;
-    if (lane == 0) kept_cnt[(size_t)s * hq + h] = count;
+    if (RULE == 2) {
+        // the lane that held the k-th largest norm owns tau
+        const uint32_t holder = __ballot_sync(0xffffffffu, tau != 0.0);
+        if (holder) tau = __shfl_sync(0xffffffffu, tau, __ffs(holder) - 1);
+    }
+    if (lane == 0) {
+        tau_out[(size_t)s * hq + h] = tau;
+        kept_cnt[(size_t)s * hq + h] = count;
+    }
 }
 
 // ---------------------------------------------------------------------------

@@ -114,6 +114,30 @@ lf_status lf_block_select(const lf_attn_desc* desc, const void* dout, const void
                           uint8_t* keep, int32_t* kept_idx, int32_t* kept_cnt,
                           void* ws, size_t ws_bytes, lf_stream_t stream);
 
+/* Selection rules of lf_block_select_rule. */
+enum {
+    LF_RULE_BUDGET = 0,          /* the LazyFlash rule of lf_block_select; param = delta in [0, 1) */
+    LF_RULE_FIXED_FRACTION = 1,  /* param = f in (0, 1]: tau = the largest threshold whose expected
+                                    kept count sum_i min(1, m_i/tau) reaches f * n (64 bisection
+                                    steps, same fixed summation order); same Philox draw and 1/p
+                                    weights as the budget rule; tau = 0 (keep all) when f = 1 */
+    LF_RULE_TOPK = 2             /* param = f in (0, 1]: keep the k = ceil(f * n) largest norms
+                                    (ties to the lower index) with weight 1, no draw; tau = the
+                                    k-th largest norm */
+};
+
+/* Block selection by one of the rules the article compares at equal backward
+ * time, "in the same CUDA implementation" (section "Le choix des blocs pèse
+ * plus que la quantité sautée"): the adaptive budget, a fraction fixed for the
+ * whole run, and top-k.  Outputs, layouts and errors are those of
+ * lf_block_select (which is rule LF_RULE_BUDGET); the backward consumes them
+ * unchanged.  LF_ERR_INVALID_ARG for an unknown rule or param out of range. */
+lf_status lf_block_select_rule(const lf_attn_desc* desc, const void* dout, const void* o,
+                               int rule, double param, uint64_t seed, uint64_t step,
+                               uint32_t flags, float* block_norm, float* D, double* tau,
+                               float* block_weight, uint8_t* keep, int32_t* kept_idx,
+                               int32_t* kept_cnt, void* ws, size_t ws_bytes, lf_stream_t stream);
+
 /* LazyFlash backward over kept query blocks (article sections "Le passage
  * arrière ..." and "Un budget sur la masse de gradient ...": dropped tiles are
  * never loaded or computed; kept blocks' output gradient is scaled by

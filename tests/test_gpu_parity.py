@@ -257,3 +257,67 @@ def test_full_size_sampled_parity(w):
         assert rel_fro(dv, dv_ref) < GRAD_TOL
     else:
         assert np.all(dk == 0) and np.all(dv == 0)
+
+
+@pytest.mark.parametrize("case", [
+    ((512,), 2, 64, 1.5),
+    ((32768,), 32, 128, 2.0),
+    ((1, 100, 0, 5000), 8, 128, 0.5),
+    ((65536,), 4, 64, 2.0),
+], ids=["tiny", "headline", "odd", "blk64_1024"])
+@pytest.mark.parametrize("rule,param", [
+    (lf.LF_RULE_FIXED_FRACTION, 0.1), (lf.LF_RULE_FIXED_FRACTION, 0.5),
+    (lf.LF_RULE_FIXED_FRACTION, 1.0), (lf.LF_RULE_TOPK, 0.1), (lf.LF_RULE_TOPK, 0.37),
+    (lf.LF_RULE_TOPK, 1.0), (lf.LF_RULE_BUDGET, 0.2),
+])
+def test_selection_rules_bit_exact_given_norms(case, rule, param):
+    """The fixed-fraction and top-k rules (article section "Le choix des blocs
+    pèse plus que la quantité sautée") in the same selection kernel."""
+    lens, hq, block, sigma = case
+    w, nb, m = _select_case(lens, hq, block, sigma, seed=7 * hq + len(lens))
+    m[0, 0, : min(3, nb[0])] = 0.0
+    m[0, 1 % hq, 5:9] = m[0, 1 % hq, 4]               # ties for top-k
+    desc = desc_for(w, torch.as_tensor(w.cu_seqlens()).cuda())
+    nbmax = w.nbmax
+    dummy = torch.zeros(w.total_tokens, hq, 64, dtype=torch.bfloat16, device="cuda")
+    norm = torch.as_tensor(m, device="cuda")
+    D = torch.empty(hq, w.total_tokens, device="cuda")
+    tau = torch.empty(w.nseq, hq, dtype=torch.float64, device="cuda")
+    wt = torch.empty(w.nseq, hq, nbmax, device="cuda")
+    keep = torch.empty(w.nseq, hq, nbmax, dtype=torch.uint8, device="cuda")
+    kidx = torch.empty(w.nseq, hq, nbmax, dtype=torch.int32, device="cuda")
+    kcnt = torch.empty(w.nseq, hq, dtype=torch.int32, device="cuda")
+    for seed, step in [(0, 0), (123, 2**33 + 5)]:
+        lf.lf_block_select_rule(desc, dummy, dummy, rule, param, seed, step, lf.LF_SELECT_NORMS_GIVEN,
+                                norm, D, tau, wt, keep, kidx, kcnt)
+        lf.lf_check_device_error()
+        ref = oracle.select_rule(rule, m, nb, param, seed, step)
+        np.testing.assert_array_equal(tau.cpu().numpy().view(np.uint64), ref["tau"].view(np.uint64))
+        np.testing.assert_array_equal(keep.cpu().numpy(), ref["keep"])
+        np.testing.assert_array_equal(wt.cpu().numpy().view(np.uint32), ref["w"].view(np.uint32))
+        np.testing.assert_array_equal(kcnt.cpu().numpy(), ref["kept_cnt"])
+        np.testing.assert_array_equal(kidx.cpu().numpy(), ref["kept_idx"])
+
+
+def test_backward_with_topk_and_fixed_fraction_weights():
+    w = synthetic.Workload("rules_bwd", (700,), hq=4, hkv=2, d=128, block=128, sigma=1.5, delta=0.1)
+    inp = synthetic.make_inputs(w)
+    dev = to_dev(inp)
+    desc = desc_for(w, dev["cu_seqlens"])
+    cu = w.cu_seqlens()
+    nb = nb_per_seq(w)
+    for rule, param in ((lf.LF_RULE_TOPK, 0.3), (lf.LF_RULE_FIXED_FRACTION, 0.4)):
+        bufs = lf.Buffers(desc)
+        lf.lf_attn_fwd(desc, dev["q"], dev["k"], dev["v"], bufs.o, bufs.lse)
+        lf.lf_block_select_rule(desc, dev["dout"], bufs.o, rule, param, 3, 1, 0, bufs.norm, bufs.D,
+                                bufs.tau, bufs.w, bufs.keep, bufs.kept_idx, bufs.kept_cnt)
+        lf.lf_attn_bwd(desc, dev["q"], dev["k"], dev["v"], bufs.o, bufs.lse, dev["dout"], bufs.D,
+                       bufs.w, bufs.kept_idx, bufs.kept_cnt, bufs.dq, bufs.dk, bufs.dv, bufs.ws)
+        lf.lf_check_device_error()
+        sel = oracle.select_rule(rule, _cpu(bufs.norm), nb, param, 3, 1)
+        np.testing.assert_array_equal(bufs.keep.cpu().numpy(), sel["keep"])
+        dq_ref, dk_ref, dv_ref = oracle.attn_bwd(cu, inp["q"], inp["k"], inp["v"], inp["dout"], w.scale,
+                                                 w.block, sel["w"].astype(np.float64), True)
+        assert rel_fro(_cpu(bufs.dq), dq_ref) < GRAD_TOL
+        assert rel_fro(_cpu(bufs.dk), dk_ref) < GRAD_TOL
+        assert rel_fro(_cpu(bufs.dv), dv_ref) < GRAD_TOL
