@@ -37,49 +37,78 @@ def build(force: bool = False) -> str:
     return _LIB
 
 
+def build_variant(mutant: int, out_path: str) -> str:
+    """Compile the oracle with planted mistake number ``mutant`` (tests only)."""
+    subprocess.check_call([
+        "gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fopenmp", "-ffp-contract=off",
+        "-fno-fast-math", "-DLFO_MUTANT=%d" % int(mutant), "-o", out_path, _SRC, "-lm",
+    ])
+    return out_path
+
+
+def use_library(path):
+    """Point this module at another build of the oracle (None: the default).
+    Returns the previous handle so that the caller can restore it."""
+    global _lib
+    with _lock:
+        prev = _lib
+        _lib = None if path is None else _declare(ctypes.CDLL(path))
+    return prev
+
+
+def restore_library(prev):
+    global _lib
+    with _lock:
+        _lib = prev
+
+
 def lib():
     global _lib
     with _lock:
         if _lib is None:
-            L = ctypes.CDLL(build())
-            dp = ctypes.POINTER(ctypes.c_double)
-            i32p = ctypes.POINTER(ctypes.c_int32)
-            u32p = ctypes.POINTER(ctypes.c_uint32)
-            c_int, c_dbl = ctypes.c_int, ctypes.c_double
-            L.lfo_philox4x32_10.argtypes = [u32p, u32p, u32p]
-            L.lfo_philox4x32_10.restype = None
-            L.lfo_block_u24.argtypes = [ctypes.c_uint64, ctypes.c_uint64, c_int, c_int, c_int]
-            L.lfo_block_u24.restype = ctypes.c_uint32
-            L.lfo_attn_fwd.argtypes = [c_int, i32p, c_int, c_int, c_int, c_int, c_dbl, c_int,
-                                       dp, dp, dp, dp, dp]
-            L.lfo_block_norms.argtypes = [c_int, i32p, c_int, c_int, c_int, c_int, c_int, dp, dp]
-            L.lfo_rowdot.argtypes = [c_int, c_int, c_int, dp, dp, dp]
-            L.lfo_pinned_sum.argtypes = [dp, c_int]
-            L.lfo_pinned_sum.restype = c_dbl
-            L.lfo_tau.argtypes = [dp, c_int, c_dbl]
-            L.lfo_tau.restype = c_dbl
-            L.lfo_discarded_mass.argtypes = [dp, c_int, c_dbl, dp]
-            L.lfo_discarded_mass.restype = c_dbl
-            L.lfo_select.argtypes = [c_int, i32p, c_int, c_int, dp, c_dbl, ctypes.c_uint64,
-                                     ctypes.c_uint64, dp, dp, ctypes.POINTER(ctypes.c_float),
-                                     ctypes.POINTER(ctypes.c_uint8), i32p, i32p]
-            L.lfo_attn_bwd.argtypes = [c_int, i32p, c_int, c_int, c_int, c_int, c_dbl, c_int,
-                                       c_int, c_int, dp, dp, dp, dp, dp, dp, dp, dp]
-            L.lfo_select_rule.argtypes = [c_int, c_int, i32p, c_int, c_int, dp, c_dbl,
-                                          ctypes.c_uint64, ctypes.c_uint64, dp, dp,
-                                          ctypes.POINTER(ctypes.c_float),
-                                          ctypes.POINTER(ctypes.c_uint8), i32p, i32p]
-            L.lfo_tau_fixed_fraction.argtypes = [dp, c_int, c_dbl]
-            L.lfo_tau_fixed_fraction.restype = c_dbl
-            L.lfo_expected_kept.argtypes = [dp, c_int, c_dbl, dp]
-            L.lfo_expected_kept.restype = c_dbl
-            L.lfo_attn_fwd_rows.argtypes = [c_int, i32p, c_int, c_int, c_int, c_int, c_dbl, c_int,
-                                            dp, dp, dp, c_int, i32p, i32p, dp, dp]
-            L.lfo_attn_bwd_rows.argtypes = [c_int, i32p, c_int, c_int, c_int, c_int, c_dbl, c_int,
-                                            c_int, c_int, dp, dp, dp, dp, dp,
-                                            c_int, i32p, i32p, dp, c_int, i32p, i32p, dp, dp]
-            _lib = L
+            _lib = _declare(ctypes.CDLL(build()))
     return _lib
+
+
+def _declare(L):
+    """Declares the C signatures on a loaded oracle library."""
+    dp = ctypes.POINTER(ctypes.c_double)
+    i32p = ctypes.POINTER(ctypes.c_int32)
+    u32p = ctypes.POINTER(ctypes.c_uint32)
+    c_int, c_dbl = ctypes.c_int, ctypes.c_double
+    L.lfo_philox4x32_10.argtypes = [u32p, u32p, u32p]
+    L.lfo_philox4x32_10.restype = None
+    L.lfo_block_u24.argtypes = [ctypes.c_uint64, ctypes.c_uint64, c_int, c_int, c_int]
+    L.lfo_block_u24.restype = ctypes.c_uint32
+    L.lfo_attn_fwd.argtypes = [c_int, i32p, c_int, c_int, c_int, c_int, c_dbl, c_int,
+                               dp, dp, dp, dp, dp]
+    L.lfo_block_norms.argtypes = [c_int, i32p, c_int, c_int, c_int, c_int, c_int, dp, dp]
+    L.lfo_rowdot.argtypes = [c_int, c_int, c_int, dp, dp, dp]
+    L.lfo_pinned_sum.argtypes = [dp, c_int]
+    L.lfo_pinned_sum.restype = c_dbl
+    L.lfo_tau.argtypes = [dp, c_int, c_dbl]
+    L.lfo_tau.restype = c_dbl
+    L.lfo_discarded_mass.argtypes = [dp, c_int, c_dbl, dp]
+    L.lfo_discarded_mass.restype = c_dbl
+    L.lfo_select.argtypes = [c_int, i32p, c_int, c_int, dp, c_dbl, ctypes.c_uint64,
+                             ctypes.c_uint64, dp, dp, ctypes.POINTER(ctypes.c_float),
+                             ctypes.POINTER(ctypes.c_uint8), i32p, i32p]
+    L.lfo_attn_bwd.argtypes = [c_int, i32p, c_int, c_int, c_int, c_int, c_dbl, c_int,
+                               c_int, c_int, dp, dp, dp, dp, dp, dp, dp, dp]
+    L.lfo_select_rule.argtypes = [c_int, c_int, i32p, c_int, c_int, dp, c_dbl,
+                                  ctypes.c_uint64, ctypes.c_uint64, dp, dp,
+                                  ctypes.POINTER(ctypes.c_float),
+                                  ctypes.POINTER(ctypes.c_uint8), i32p, i32p]
+    L.lfo_tau_fixed_fraction.argtypes = [dp, c_int, c_dbl]
+    L.lfo_tau_fixed_fraction.restype = c_dbl
+    L.lfo_expected_kept.argtypes = [dp, c_int, c_dbl, dp]
+    L.lfo_expected_kept.restype = c_dbl
+    L.lfo_attn_fwd_rows.argtypes = [c_int, i32p, c_int, c_int, c_int, c_int, c_dbl, c_int,
+                                    dp, dp, dp, c_int, i32p, i32p, dp, dp]
+    L.lfo_attn_bwd_rows.argtypes = [c_int, i32p, c_int, c_int, c_int, c_int, c_dbl, c_int,
+                                    c_int, c_int, dp, dp, dp, dp, dp,
+                                    c_int, i32p, i32p, dp, c_int, i32p, i32p, dp, dp]
+    return L
 
 
 def _f64(a) -> np.ndarray:

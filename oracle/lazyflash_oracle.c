@@ -46,6 +46,13 @@
 #define LFO_OK 0
 #define LFO_EINVAL 1
 
+/* LFO_MUTANT selects one deliberately planted mistake, so that the tests can
+ * check that the pins catch it (tests/test_oracle_mutants.py).  0 = the
+ * oracle as written; every other value is used only by that test. */
+#ifndef LFO_MUTANT
+#define LFO_MUTANT 0
+#endif
+
 /* ------------------------------------------------------------------------ */
 /* Philox4x32-10 (Salmon et al., SC'11, section 5): a 10-round bijection of a  */
 /* 128-bit counter under a 64-bit key.  Each round multiplies words 0 and 2 by */
@@ -61,7 +68,7 @@ void lfo_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t ou
 {
     uint32_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3];
     uint32_t k0 = key[0], k1 = key[1];
-    for (int round = 0; round < 10; ++round) {
+    for (int round = 0; round < (LFO_MUTANT == 7 ? 9 : 10); ++round) {
         if (round > 0) { k0 += PHILOX_W0; k1 += PHILOX_W1; }
         uint64_t p0 = (uint64_t)PHILOX_M0 * (uint64_t)c0;
         uint64_t p1 = (uint64_t)PHILOX_M1 * (uint64_t)c2;
@@ -95,15 +102,15 @@ uint32_t lfo_block_u24(uint64_t seed, uint64_t step, int s, int h, int i)
 static int row_scores(int t, int seg0, int seg1, int causal, int hq, int hkv, int d,
                       double scale, int h, const double* q, const double* k, double* srow)
 {
-    int G = hq / hkv, g = h / G;
-    int u_end = causal ? t + 1 : seg1;
+    int G = hq / hkv, g = (LFO_MUTANT == 2) ? h % hkv : h / G;
+    int u_end = causal ? ((LFO_MUTANT == 9 && t > seg0) ? t : t + 1) : seg1;
     const double* qt = q + ((size_t)t * hq + h) * d;
     int n = 0;
     for (int u = seg0; u < u_end; ++u) {
         const double* ku = k + ((size_t)u * hkv + g) * d;
         double acc = 0.0;
         for (int c = 0; c < d; ++c) acc += qt[c] * ku[c];
-        srow[n++] = scale * acc;
+        srow[n++] = (LFO_MUTANT == 1) ? acc : scale * acc;
     }
     return n;
 }
@@ -192,7 +199,7 @@ int lfo_block_norms(int nseq, const int32_t* cu, int T, int hq, int d, int block
                         for (int c = 0; c < d; ++c) acc += row[c] * row[c];
                     }
                 }
-                norms[((size_t)s * hq + h) * nbmax + i] = sqrt(acc);
+                norms[((size_t)s * hq + h) * nbmax + i] = (LFO_MUTANT == 10) ? acc : sqrt(acc);
             }
         }
     return LFO_OK;
@@ -236,7 +243,8 @@ double lfo_pinned_sum(const double* x, int n)
 double lfo_discarded_mass(const double* m, int n, double tau, double* scratch)
 {
     for (int b = 0; b < n; ++b)
-        scratch[b] = (m[b] >= tau) ? 0.0 : (1.0 - m[b] / tau) * m[b];
+        scratch[b] = (m[b] >= tau) ? 0.0
+                   : (LFO_MUTANT == 6 ? (m[b] / tau) * m[b] : (1.0 - m[b] / tau) * m[b]);
     return lfo_pinned_sum(scratch, n);
 }
 
@@ -296,7 +304,7 @@ int lfo_select(int nseq, const int32_t* nb, int hq, int nbmax, const double* nor
                         uint32_t u = lfo_block_u24(seed, step, s, h, i);
                         kb = ((double)u < pi * 16777216.0);
                     }
-                    if (kb) wi = (float)(1.0 / pi);
+                    if (kb) wi = (float)(LFO_MUTANT == 8 ? pi : 1.0 / pi);
                 }
                 p[base + i] = pi;
                 keep[base + i] = (uint8_t)kb;
@@ -353,7 +361,8 @@ int lfo_attn_bwd(int nseq, const int32_t* cu, int T, int hq, int hkv, int d, dou
                             for (int c = 0; c < d; ++c) ot[c] += prow[i] * vu[c];
                         }
                         double Dt = 0.0;
-                        for (int c = 0; c < d; ++c) Dt += dot_[c] * ot[c];
+                        for (int c = 0; c < d; ++c)
+                            Dt += (LFO_MUTANT == 3 ? dot_raw[c] : dot_[c]) * ot[c];
                         const double* qt = q + ((size_t)t * hq + h) * d;
                         double* dqt = dq + ((size_t)t * hq + h) * d;
                         for (int i = 0; i < n; ++i) {
@@ -363,12 +372,12 @@ int lfo_attn_bwd(int nseq, const int32_t* cu, int T, int hq, int hkv, int d, dou
                             double dP = 0.0;
                             for (int c = 0; c < d; ++c) dP += dot_[c] * vu[c];
                             double P = prow[i];
-                            double dS = P * (dP - Dt);
+                            double dS = (LFO_MUTANT == 5) ? P * (Dt - dP) : P * (dP - Dt);
                             double* dku = dk + ((size_t)u * hkv + g) * d;
                             double* dvu = dv + ((size_t)u * hkv + g) * d;
                             for (int c = 0; c < d; ++c) {
                                 dqt[c] += scale * dS * ku[c];
-                                dku[c] += scale * dS * qt[c];
+                                dku[c] += (LFO_MUTANT == 4 ? 1.0 : scale) * dS * qt[c];
                                 dvu[c] += P * dot_[c];
                             }
                         }
