@@ -21,10 +21,10 @@
 //   tcgen05 (SS): dQ_h^T = K_j^T dS^T_h                  (TMEM, lanes = d)
 //   dQ drain:     lane d adds column q of dQ_h^T into the fp32 accumulator;
 //                 a warp's 32 lanes hit 32 consecutive floats of one row.
-// Roles (512 threads): warp 0 TMA producer and work list, warp 1 MMA issuer,
-// warps 4-7 element-wise half 0 (+ dV epilogue), warps 12-15 element-wise
-// half 1 (+ dK epilogue): thread = KV row = TMEM lane; warps 8-11 dQ drain
-// (thread = head-dim index = TMEM lane).
+// Roles (512 threads): warp 0 TMA producer and work list, warp 1 MMA issuer (the
+// whole warp runs it, one elected lane issues), warps 4-7 element-wise half 0
+// (+ dV epilogue), warps 12-15 element-wise half 1 (+ dK epilogue): thread = KV
+// row = TMEM lane; warps 8-11 dQ drain (thread = head-dim index = TMEM lane).
 //
 // Tensor memory (512 columns): dV [0,128) dK [128,256); half 0: S^T/P^T/dQ^T
 // [256,320), dP^T/dS^T [320,384); half 1: [384,448), [448,512).  Reuse of a
@@ -281,23 +281,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         }
         __syncwarp();
     } else if (warp == 1) {
-        // ===================== MMA issuer (one thread) =====================
-        if (lane == 0 && any) {
+        // ============ MMA issuer: the whole warp, one elected lane issues ============
+        // (issuing from converged code keeps the tensor pipe fed; every wait result is
+        // made warp-uniform, and each commit tracks the MMAs of the issuing lane)
+        if (any) {
+            auto wait = [&](uint64_t* bar, uint32_t parity, int site) {
+                return __all_sync(0xffffffffu, mbar_wait_or_abort(bar, parity, site, abort_flag));
+            };
             const uint32_t ka = s_base + L::kK, va = s_base + L::kV;
-            const bool ok = mbar_wait_or_abort(bar_kv, 0, 33, abort_flag);
+            const bool ok = wait(bar_kv, 0, 33);
             int n = 0;
             bool more = ok;
             while (more) {
                 const int st = n & 1;
-                if (!mbar_wait_or_abort(&bar_entry[n & 3], (n >> 2) & 1, 34, abort_flag)) break;
+                if (!wait(&bar_entry[n & 3], (n >> 2) & 1, 34)) break;
                 if (ring[n & 3].h < 0) break;
-                if (!mbar_wait_or_abort(&bar_qdo_full[st], (n >> 1) & 1, 34, abort_flag)) break;
+                if (!wait(&bar_qdo_full[st], (n >> 1) & 1, 34)) break;
                 const uint32_t qa = s_base + L::kQdo + (2 * st) * L::kTile;
                 const uint32_t da = qa + L::kTile;
                 // S^T and dP^T of both halves
                 bool w_ok = true;
                 for (int hf = 0; hf < 2; ++hf) {
-                    if (n > 0 && !mbar_wait_or_abort(&bar_dq_free[hf], (n - 1) & 1, 35, abort_flag)) {
+                    if (n > 0 && !wait(&bar_dq_free[hf], (n - 1) & 1, 35)) {
                         w_ok = false;
                         break;
                     }
@@ -305,16 +310,16 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     const uint32_t t_s = tmem + 256 + hf * 128, t_dp = t_s + 64;
 #pragma unroll
                     for (int k = 0; k < D / 16; ++k)
-                        mma_bf16_ss(t_s, desc_kmajor(ka, k), desc_kmajor(qa + hf * 8192, k), kIdescS, k > 0);
+                        mma_bf16_ss_warp(t_s, desc_kmajor(ka, k), desc_kmajor(qa + hf * 8192, k), kIdescS, k > 0);
 #pragma unroll
                     for (int k = 0; k < D / 16; ++k)
-                        mma_bf16_ss(t_dp, desc_kmajor(va, k), desc_kmajor(da + hf * 8192, k), kIdescS, k > 0);
-                    mma_commit(&bar_s_full[hf]);
+                        mma_bf16_ss_warp(t_dp, desc_kmajor(va, k), desc_kmajor(da + hf * 8192, k), kIdescS, k > 0);
+                    mma_commit_warp(&bar_s_full[hf]);
                 }
                 if (!w_ok) break;
                 // dV, dK (TS) and dQ^T (SS) of both halves
                 for (int hf = 0; hf < 2; ++hf) {
-                    if (!mbar_wait_or_abort(&bar_p_ready[hf], n & 1, 36, abort_flag)) {
+                    if (!wait(&bar_p_ready[hf], n & 1, 36)) {
                         w_ok = false;
                         break;
                     }
@@ -322,13 +327,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     const uint32_t t_s = tmem + 256 + hf * 128, t_dp = t_s + 64;
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
-                        mma_bf16_ts(t_dv, t_s + k * 8, desc_mnmajor(da, hf * 4 + k), kIdescKV,
-                                    (n > 0 || hf > 0 || k > 0) ? 1u : 0u);
+                        mma_bf16_ts_warp(t_dv, t_s + k * 8, desc_mnmajor(da, hf * 4 + k), kIdescKV,
+                                         (n > 0 || hf > 0 || k > 0) ? 1u : 0u);
 #pragma unroll
                     for (int k = 0; k < 4; ++k)
-                        mma_bf16_ts(t_dk, t_dp + k * 8, desc_mnmajor(qa, hf * 4 + k), kIdescKV,
-                                    (n > 0 || hf > 0 || k > 0) ? 1u : 0u);
-                    if (hf == 1) mma_commit(&bar_qdo_empty[st]);   // Q/dO of this stage fully read
+                        mma_bf16_ts_warp(t_dk, t_dp + k * 8, desc_mnmajor(qa, hf * 4 + k), kIdescKV,
+                                         (n > 0 || hf > 0 || k > 0) ? 1u : 0u);
+                    if (hf == 1) mma_commit_warp(&bar_qdo_empty[st]);   // Q/dO of this stage fully read
                     const uint32_t dsa = s_base + L::kDS + hf * L::kHalfDS;
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
@@ -336,18 +341,17 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         // second 64-row atom repeats the first (those lanes are unused)
                         const uint64_t adesc =
                             (D == 128) ? desc_mnmajor(ka, k) : sw128_desc(ka + k * 2048, 0, 1024);
-                        mma_bf16_ss(t_s, adesc, desc_mnmajor(dsa, k), kIdescQ, k > 0);
+                        mma_bf16_ss_warp(t_s, adesc, desc_mnmajor(dsa, k), kIdescQ, k > 0);
                     }
-                    mma_commit(&bar_dq_full[hf]);
+                    mma_commit_warp(&bar_dq_full[hf]);
                 }
                 if (!w_ok) break;
                 ++n;
             }
-            mma_commit(bar_done);
-            // every MMA this thread issued must finish before TMEM is released
-            mbar_wait(bar_done, 0, 37);
+            mma_commit_warp(bar_done);
+            // every MMA this warp issued must finish before TMEM is released
+            __all_sync(0xffffffffu, mbar_wait(bar_done, 0, 37));
         }
-        __syncwarp();
     } else if ((warp >= 4 && warp < 8) || warp >= 12) {
         // ===== element-wise: both warpgroups on each half, 32 columns each (thread = KV row) =====
         const int wg = warp >= 12 ? 1 : 0;                // columns [32 wg, 32 wg + 32) of a half

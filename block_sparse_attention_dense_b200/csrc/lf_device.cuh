@@ -155,6 +155,40 @@ __device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, ui
         : "memory");
 }
 
+// Warp-wide forms of the MMA issue and commit: the whole warp executes them and one
+// elected lane issues.  Issuing from converged code keeps the descriptors warp-uniform,
+// which roughly halves the time a warp needs to issue one MMA (a single-lane issue costs
+// about as long as a 128x128x16 MMA takes to run, so the tensor pipe would starve).
+__device__ __forceinline__ void mma_bf16_ss_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                 uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\t"
+        "elect.sync r|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+__device__ __forceinline__ void mma_bf16_ts_warp(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                 uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p, e;\n\t.reg .b32 r;\n\t"
+        "elect.sync r|e, 0xffffffff;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+// One arrival on `bar` (from the elected lane) once every MMA the warp issued has completed.
+__device__ __forceinline__ void mma_commit_warp(uint64_t* bar) {
+    asm volatile(
+        "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
+        "elect.sync r|e, 0xffffffff;\n\t"
+        "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
+            smem_addr(bar))
+        : "memory");
+}
+
 // Arrive once on `bar` when every MMA this thread issued so far has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
     asm volatile(
@@ -285,6 +319,26 @@ __device__ __forceinline__ float fast_exp2(float x) {
     return y;
 }
 
+// Per-warpgroup register budgets (setmaxnreg): every thread of the warpgroup executes
+// the same call.  An increase waits until other warpgroups have released enough of the
+// registers the block was launched with, so the budgets after the change must add up to
+// no more than that launch total.
+template <uint32_t N>
+__device__ __forceinline__ void regs_release_to() {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+template <uint32_t N>
+__device__ __forceinline__ void regs_grow_to() {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;\n" ::"n"(N));
+}
+
+// max(a, b, c) in one instruction (sm_100 three-input form).
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+    float r;
+    asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+
 }  // namespace lf
 
 namespace lf {
@@ -356,6 +410,17 @@ __device__ __forceinline__ bool named_bar_or(int id, int nthreads, bool v) {
 namespace lf {
 
 // 16 consecutive 32-bit TMEM columns of this thread's lane, without waiting.
+// Ties 16 load destinations to a preceding tmem_wait_ld(), so that no use of them is
+// scheduled before the wait.
+__device__ __forceinline__ void tmem_regs_ready(uint32_t (&r)[16]) {
+    asm volatile(""
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+                   "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]),
+                   "+r"(r[13]), "+r"(r[14]), "+r"(r[15])
+                 :
+                 : "memory");
+}
+
 // The registers are valid only after tmem_wait_ld_regs() on them.
 __device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
@@ -416,6 +481,23 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&v)[8])
         "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(taddr),
         "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
         : "memory");
+}
+
+// Bounded spin until the shared-memory counter *seq reaches `need` (a plain volatile
+// poll: the wait is short and a suspended warp would wake later than a poll).
+__device__ __forceinline__ bool spin_until_geq(const volatile int* seq, int need, int site,
+                                               volatile int* abort) {
+    if (*seq >= need) return true;
+    const long long t0 = clock64();
+    for (;;) {
+        if (*seq >= need) return true;
+        if (*abort) return false;
+        if (clock64() - t0 > kWaitLimitCycles) {
+            report_timeout(site);
+            *abort = 1;
+            return false;
+        }
+    }
 }
 
 }  // namespace lf

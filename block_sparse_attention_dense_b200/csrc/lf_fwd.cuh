@@ -21,6 +21,8 @@
 // of a region by a later MMA relies on tcgen05.mma executing in issue order.
 #pragma once
 
+#include <climits>
+
 #include "lf_device.cuh"
 
 namespace lf {
@@ -46,6 +48,9 @@ struct FwdSmem {
 };
 
 constexpr int kFwdThreads = 384;
+constexpr int kFwdLaunchRegs = 168;     // 65536 / 384, rounded down to a multiple of 8
+constexpr int kFwdCtrlRegs = 64;
+constexpr int kFwdSoftmaxRegs = 216;
 constexpr float kRescaleThreshold = 8.0f;   // log2 of the largest P before a rescale
 
 template <int D>
@@ -64,9 +69,10 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     uint64_t* bar_s_full = bars + 9;    // [2] per query tile
     uint64_t* bar_p_ready = bars + 11;  // [2]
     uint64_t* bar_o_done = bars + 13;   // [2]
-    uint64_t* bar_done = bars + 15;
-    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 16);
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 17);
+    uint64_t* bar_done = bars + 15;     // [2] per MMA issuer
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 18);
+    volatile int* burst_seq = reinterpret_cast<volatile int*>(bars + 19);   // [2] bursts issued per MMA issuer
 
     const int h = blockIdx.y;
     const int s = blockIdx.z;
@@ -90,15 +96,18 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
         mbar_init(bar_q, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bar_k_full[i], 1);
-            mbar_init(&bar_k_empty[i], 1);
+            mbar_init(&bar_k_empty[i], two ? 2 : 1);   // one commit per query tile
             mbar_init(&bar_v_full[i], 1);
-            mbar_init(&bar_v_empty[i], 1);
+            mbar_init(&bar_v_empty[i], two ? 2 : 1);
             mbar_init(&bar_s_full[i], 1);
             mbar_init(&bar_p_ready[i], 128);
             mbar_init(&bar_o_done[i], 1);
         }
-        mbar_init(bar_done, 1);
+        mbar_init(&bar_done[0], 1);
+        mbar_init(&bar_done[1], 1);
         *abort_flag = 0;
+        burst_seq[0] = 0;
+        burst_seq[1] = two ? 0 : INT_MAX;   // a lone tile never waits for its turn
         fence_barrier_init();
         prefetch_tensormap(&tm_q);
         prefetch_tensormap(&tm_k);
@@ -112,103 +121,113 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-
-    if (warp == 0) {
-        // ===================== TMA producer =====================
-        if (lane == 0) {
-            const uint32_t qbytes = (two ? 2 : 1) * L::kTile;
-            mbar_arrive_expect_tx(bar_q, qbytes);
-            for (int t = 0; t < (two ? 2 : 1); ++t)
-                for (int c = 0; c < L::kPanels; ++c)
-                    tma_load_3d(smem + L::kQ + t * L::kTile + c * kPanelBytes, &tm_q, bar_q, c * 64, h,
-                                seg0 + (2 * m + t) * 128);
-            uint32_t kpar[2] = {0, 0}, vpar[2] = {0, 0};
-            int kfill = 0, vfill = 0;   // loads issued (for the drain on abort)
-            for (int j = 0; j < nkv; ++j) {
-                const int st = j & 1;
-                if (j >= 2 && !mbar_wait_or_abort(&bar_k_empty[st], ((j >> 1) - 1) & 1, 21, abort_flag)) break;
-                mbar_arrive_expect_tx(&bar_k_full[st], L::kTile);
-                for (int c = 0; c < L::kPanels; ++c)
-                    tma_load_3d(smem + L::kK + st * L::kTile + c * kPanelBytes, &tm_k, &bar_k_full[st],
-                                c * 64, g, seg0 + j * 128);
-                kpar[st] = (j >> 1) & 1;
-                ++kfill;
-                if (j >= 2 && !mbar_wait_or_abort(&bar_v_empty[st], ((j >> 1) - 1) & 1, 22, abort_flag)) break;
-                mbar_arrive_expect_tx(&bar_v_full[st], L::kTile);
-                for (int c = 0; c < L::kPanels; ++c)
-                    tma_load_3d(smem + L::kV + st * L::kTile + c * kPanelBytes, &tm_v, &bar_v_full[st],
-                                c * 64, g, seg0 + j * 128);
-                vpar[st] = (j >> 1) & 1;
-                ++vfill;
-            }
-            if (*abort_flag) {
-                // let this CTA's own copies land before the CTA exits (bounded)
-                mbar_wait(bar_q, 0, 23);
-                for (int st = 0; st < 2; ++st) {
-                    if (kfill > st) mbar_wait(&bar_k_full[st], kpar[st], 23);
-                    if (vfill > st) mbar_wait(&bar_v_full[st], vpar[st], 23);
+    // 384 threads x 168 registers at launch >= 128 x 64 (TMA, MMA, idle) + 256 x 216 (softmax)
+    static_assert(128 * kFwdCtrlRegs + 256 * kFwdSoftmaxRegs <= kFwdThreads * kFwdLaunchRegs, "register split");
+    if (warp < 4) {
+        regs_release_to<kFwdCtrlRegs>();
+        if (warp == 0) {
+            // ===================== TMA producer =====================
+            if (lane == 0) {
+                const uint32_t qbytes = (two ? 2 : 1) * L::kTile;
+                mbar_arrive_expect_tx(bar_q, qbytes);
+                for (int t = 0; t < (two ? 2 : 1); ++t)
+                    for (int c = 0; c < L::kPanels; ++c)
+                        tma_load_3d(smem + L::kQ + t * L::kTile + c * kPanelBytes, &tm_q, bar_q, c * 64, h,
+                                    seg0 + (2 * m + t) * 128);
+                uint32_t kpar[2] = {0, 0}, vpar[2] = {0, 0};
+                int kfill = 0, vfill = 0;   // loads issued (for the drain on abort)
+                for (int j = 0; j < nkv; ++j) {
+                    const int st = j & 1;
+                    if (j >= 2 && !mbar_wait_or_abort(&bar_k_empty[st], ((j >> 1) - 1) & 1, 21, abort_flag)) break;
+                    mbar_arrive_expect_tx(&bar_k_full[st], L::kTile);
+                    for (int c = 0; c < L::kPanels; ++c)
+                        tma_load_3d(smem + L::kK + st * L::kTile + c * kPanelBytes, &tm_k, &bar_k_full[st],
+                                    c * 64, g, seg0 + j * 128);
+                    kpar[st] = (j >> 1) & 1;
+                    ++kfill;
+                    if (j >= 2 && !mbar_wait_or_abort(&bar_v_empty[st], ((j >> 1) - 1) & 1, 22, abort_flag)) break;
+                    mbar_arrive_expect_tx(&bar_v_full[st], L::kTile);
+                    for (int c = 0; c < L::kPanels; ++c)
+                        tma_load_3d(smem + L::kV + st * L::kTile + c * kPanelBytes, &tm_v, &bar_v_full[st],
+                                    c * 64, g, seg0 + j * 128);
+                    vpar[st] = (j >> 1) & 1;
+                    ++vfill;
+                }
+                if (*abort_flag) {
+                    // let this CTA's own copies land before the CTA exits (bounded)
+                    mbar_wait(bar_q, 0, 23);
+                    for (int st = 0; st < 2; ++st) {
+                        if (kfill > st) mbar_wait(&bar_k_full[st], kpar[st], 23);
+                        if (vfill > st) mbar_wait(&bar_v_full[st], vpar[st], 23);
+                    }
                 }
             }
-        }
-        __syncwarp();
-    } else if (warp == 1) {
-        // ===================== MMA issuer (one thread) =====================
-        if (lane == 0) {
-            constexpr uint32_t kIdescS = idesc_bf16(128, 128, 0, 0);
-            constexpr uint32_t kIdescO = idesc_bf16(128, D, 0, 1);
-            const uint32_t qa0 = s_base + L::kQ;
-            auto issue_s = [&](int t, int j) {
-                const uint32_t qa = qa0 + t * L::kTile;
-                const uint32_t ka = s_base + L::kK + (j & 1) * L::kTile;
+            __syncwarp();
+        } else if (warp == 1 || warp == 2) {
+            // ============ MMA issuers: warp 1 for query tile 0, warp 2 for tile 1 ============
+            // The tensor pipe sees the bursts in the single-issuer order S0 S1 | PV0 S0' |
+            // PV1 S1' | ..., so each tile's softmax overlaps the other tile's MMAs, but each
+            // issuer clears its own barrier waits while the other one's burst runs.  A burst
+            // waits for its turn on the other issuer's count of bursts issued.  The whole
+            // warp runs this code (one elected lane issues); every wait result is made
+            // warp-uniform.  Each commit tracks only the MMAs of the issuing lane.
+            const int t = warp - 1;
+            const int nk = t ? nkv1 : nkv0;
+            if (nk > 0) {
+                constexpr uint32_t kIdescS = idesc_bf16(128, 128, 0, 0);
+                constexpr uint32_t kIdescO = idesc_bf16(128, D, 0, 1);
+                const uint32_t qa = s_base + L::kQ + t * L::kTile;
+                const uint32_t t_s = tmem + t * 128, t_o = tmem + 256 + t * 128;
+                int nb = 0;   // bursts this warp has issued
+                auto wait = [&](uint64_t* bar, uint32_t parity, int site) {
+                    return __all_sync(0xffffffffu, mbar_wait_or_abort(bar, parity, site, abort_flag));
+                };
+                auto my_turn = [&]() {
+                    return __all_sync(0xffffffffu, spin_until_geq(&burst_seq[1 - t], nb + t, 19, abort_flag));
+                };
+                auto publish = [&](int v) {
+                    __syncwarp();
+                    if (lane == 0) burst_seq[t] = v;
+                    __syncwarp();
+                };
+                auto issue_s = [&](int j) {
+                    const uint32_t ka = s_base + L::kK + (j & 1) * L::kTile;
 #pragma unroll
-                for (int k = 0; k < D / 16; ++k)
-                    mma_bf16_ss(tmem + t * 128, desc_kmajor(qa, k), desc_kmajor(ka, k), kIdescS, k > 0);
-                mma_commit(&bar_s_full[t]);
-            };
-            bool ok = mbar_wait_or_abort(bar_q, 0, 24, abort_flag) &&
-                      mbar_wait_or_abort(&bar_k_full[0], 0, 25, abort_flag);
-            if (ok) {
-                tc_fence_after();
-                issue_s(0, 0);
-                if (two) issue_s(1, 0);
-                mma_commit(&bar_k_empty[0]);
-            }
-            for (int j = 0; j < nkv && ok; ++j) {
-                const int st = j & 1;
-                if (!mbar_wait_or_abort(&bar_v_full[st], (j >> 1) & 1, 26, abort_flag)) break;
-                bool k_next_ready = false;
-                for (int t = 0; t < 2; ++t) {
-                    const int nk = t ? nkv1 : nkv0;
-                    if (j >= nk) continue;
-                    if (!mbar_wait_or_abort(&bar_p_ready[t], j & 1, 27, abort_flag)) { ok = false; break; }
+                    for (int k = 0; k < D / 16; ++k)
+                        mma_bf16_ss_warp(t_s, desc_kmajor(qa, k), desc_kmajor(ka, k), kIdescS, k > 0);
+                    mma_commit_warp(&bar_s_full[t]);
+                    mma_commit_warp(&bar_k_empty[j & 1]);
+                };
+                bool ok = wait(bar_q, 0, 24) && wait(&bar_k_full[0], 0, 25) && my_turn();
+                if (ok) {
+                    tc_fence_after();
+                    issue_s(0);
+                    publish(++nb);
+                }
+                for (int j = 0; j < nk && ok; ++j) {
+                    const int st = j & 1;
+                    if (!wait(&bar_v_full[st], (j >> 1) & 1, 26)) break;
+                    if (!wait(&bar_p_ready[t], j & 1, 27)) break;
+                    if (j + 1 < nk && !wait(&bar_k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, 28)) break;
+                    if (!my_turn()) break;
                     tc_fence_after();
                     const uint32_t va = s_base + L::kV + st * L::kTile;
 #pragma unroll
                     for (int k = 0; k < 8; ++k)
-                        mma_bf16_ts(tmem + 256 + t * 128, tmem + t * 128 + k * 8, desc_mnmajor(va, k),
-                                    kIdescO, (j > 0 || k > 0) ? 1u : 0u);
-                    mma_commit(&bar_o_done[t]);
-                    if (j + 1 < nk) {
-                        if (!k_next_ready) {
-                            if (!mbar_wait_or_abort(&bar_k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, 28, abort_flag)) {
-                                ok = false;
-                                break;
-                            }
-                            tc_fence_after();
-                            k_next_ready = true;
-                        }
-                        issue_s(t, j + 1);
-                    }
+                        mma_bf16_ts_warp(t_o, t_s + k * 8, desc_mnmajor(va, k), kIdescO, (j > 0 || k > 0) ? 1u : 0u);
+                    mma_commit_warp(&bar_o_done[t]);
+                    mma_commit_warp(&bar_v_empty[st]);
+                    if (j + 1 < nk) issue_s(j + 1);
+                    publish(++nb);
                 }
-                if (!ok) break;
-                mma_commit(&bar_v_empty[st]);
-                if (k_next_ready) mma_commit(&bar_k_empty[(j + 1) & 1]);
+                publish(INT_MAX);   // finished (or aborted): never hold the other issuer
+                mma_commit_warp(&bar_done[t]);
+                // every MMA issued by this warp has finished (waits even after an abort)
+                __all_sync(0xffffffffu, mbar_wait(&bar_done[t], 0, 29));
             }
-            mma_commit(bar_done);
-            mbar_wait(bar_done, 0, 29);   // every MMA issued here has finished
         }
-        __syncwarp();
-    } else if (warp >= 4 && warp < 12) {
+    } else {
+        regs_grow_to<kFwdSoftmaxRegs>();
         // ============ softmax, one warpgroup per query tile (thread = row) ============
         const int t = (warp - 4) >> 2;
         const int r = (warp & 3) * 32 + lane;
@@ -224,40 +243,40 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             const bool got = mbar_wait_or_abort(&bar_s_full[t], j & 1, 30, abort_flag);
             if (!__all_sync(0xffffffffu, got)) { failed = true; break; }
             tc_fence_after();
+            // the row's 128 score columns: eight loads in flight, one wait
             float sv[128];
             {
-                uint32_t a[16], b[16];
+                uint32_t sr[8][16];
 #pragma unroll
-                for (int c = 0; c < 8; c += 2) {
-                    tmem_ld16_nowait(t_s + c * 16, a);
-                    tmem_ld16_nowait(t_s + (c + 1) * 16, b);
-                    tmem_wait_ld_regs(a, b);
+                for (int c = 0; c < 8; ++c) tmem_ld16_nowait(t_s + c * 16, sr[c]);
+                tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        sv[c * 16 + e] = __uint_as_float(a[e]);
-                        sv[(c + 1) * 16 + e] = __uint_as_float(b[e]);
-                    }
+                for (int c = 0; c < 8; ++c) {
+                    tmem_regs_ready(sr[c]);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) sv[c * 16 + e] = __uint_as_float(sr[c][e]);
                 }
             }
             const int kv0 = j * 128;
             const bool diag = prm.causal && j == qt;
             const bool tail = kv0 + 128 > len;
-            float mx = -INFINITY;
             if (diag || tail) {
 #pragma unroll
                 for (int e = 0; e < 128; ++e) {
                     const int kv = kv0 + e;
                     const bool valid = !(diag && kv > q_local) && kv < len;
-                    sv[e] = valid ? sv[e] * prm.scale_log2 : -INFINITY;
-                    mx = fmaxf(mx, sv[e]);
-                }
-            } else {
-#pragma unroll
-                for (int e = 0; e < 128; ++e) {
-                    sv[e] *= prm.scale_log2;
-                    mx = fmaxf(mx, sv[e]);
+                    sv[e] = valid ? sv[e] : -INFINITY;
                 }
             }
+            // row maximum of the raw scores (three-input maxima, four independent chains);
+            // the scale is positive, so scaling the maximum gives the scaled maximum
+            float mq[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+            for (int e = 0; e < 128; e += 8) {
+#pragma unroll
+                for (int q = 0; q < 4; ++q) mq[q] = fmax3(mq[q], sv[e + 2 * q], sv[e + 2 * q + 1]);
+            }
+            const float mx = fmax3(mq[0], mq[1], fmaxf(mq[2], mq[3])) * prm.scale_log2;
             // stale-max rule: keep the old reference unless the row maximum grew a lot
             float alpha = 1.f;
             bool rescale = false;
@@ -268,20 +287,38 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 m_ref = mx;
                 rescale = true;
             }
-            float rs = 0.f;
+            // P = 2^(scale * S - m_ref), in four chunks of 32 columns, software-pipelined:
+            // the exponentials of chunk c+1 are issued ahead of the row sums, the bf16
+            // packing and the TMEM store of chunk c, so that one warp keeps the MUFU busy
+            const float neg_m = -m_ref;
+            float rs[4] = {0.f, 0.f, 0.f, 0.f};
+            auto exps = [&](int c, float (&p)[32]) {
 #pragma unroll
-            for (int c = 0; c < 4; ++c) {
+                for (int e = 0; e < 32; ++e) p[e] = fast_exp2(fmaf(sv[c * 32 + e], prm.scale_log2, neg_m));
+            };
+            auto finish = [&](int c, const float (&p)[32]) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    const float p0 = fast_exp2(sv[c * 32 + 2 * e] - m_ref);
-                    const float p1 = fast_exp2(sv[c * 32 + 2 * e + 1] - m_ref);
-                    rs += p0 + p1;
-                    pk[e] = pack_bf16(p0, p1);
+                    rs[(e & 1) * 2] += p[2 * e];
+                    rs[(e & 1) * 2 + 1] += p[2 * e + 1];
+                    pk[e] = pack_bf16(p[2 * e], p[2 * e + 1]);
                 }
                 tmem_st16(t_s + c * 16, pk);   // P (packed) over S columns already read
+            };
+            {
+                float pa[32], pb[32];
+                exps(0, pa);
+                exps(1, pb);
+                finish(0, pa);
+                exps(2, pa);
+                finish(1, pb);
+                exps(3, pb);
+                finish(2, pa);
+                finish(3, pb);
             }
-            l_run = l_run * alpha + rs;
+            const float rs_all = (rs[0] + rs[1]) + (rs[2] + rs[3]);
+            l_run = l_run * alpha + rs_all;
             if (__any_sync(0xffffffffu, rescale)) {
                 // O_t must hold the previous P.V product before it is rescaled
                 const bool got_o = mbar_wait_or_abort(&bar_o_done[t], (j - 1) & 1, 31, abort_flag);
