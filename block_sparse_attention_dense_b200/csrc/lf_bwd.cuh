@@ -289,64 +289,74 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 return __all_sync(0xffffffffu, mbar_wait_or_abort(bar, parity, site, abort_flag));
             };
             const uint32_t ka = s_base + L::kK, va = s_base + L::kV;
-            const bool ok = wait(bar_kv, 0, 33);
-            int n = 0;
-            bool more = ok;
-            while (more) {
-                const int st = n & 1;
-                if (!wait(&bar_entry[n & 3], (n >> 2) & 1, 34)) break;
-                if (ring[n & 3].h < 0) break;
-                if (!wait(&bar_qdo_full[st], (n >> 1) & 1, 34)) break;
-                const uint32_t qa = s_base + L::kQdo + (2 * st) * L::kTile;
-                const uint32_t da = qa + L::kTile;
-                // S^T and dP^T of both halves
-                bool w_ok = true;
-                for (int hf = 0; hf < 2; ++hf) {
-                    if (n > 0 && !wait(&bar_dq_free[hf], (n - 1) & 1, 35)) {
-                        w_ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    const uint32_t t_s = tmem + 256 + hf * 128, t_dp = t_s + 64;
+            auto stage_q = [&](int n) { return s_base + L::kQdo + (2 * (n & 1)) * L::kTile; };
+            // S^T and dP^T of one half of pair n
+            auto issue_sdp = [&](int hf, int n) {
+                const uint32_t qa = stage_q(n), da = qa + L::kTile;
+                const uint32_t t_s = tmem + 256 + hf * 128, t_dp = t_s + 64;
 #pragma unroll
-                    for (int k = 0; k < D / 16; ++k)
-                        mma_bf16_ss_warp(t_s, desc_kmajor(ka, k), desc_kmajor(qa + hf * 8192, k), kIdescS, k > 0);
+                for (int k = 0; k < D / 16; ++k)
+                    mma_bf16_ss_warp(t_s, desc_kmajor(ka, k), desc_kmajor(qa + hf * 8192, k), kIdescS, k > 0);
 #pragma unroll
-                    for (int k = 0; k < D / 16; ++k)
-                        mma_bf16_ss_warp(t_dp, desc_kmajor(va, k), desc_kmajor(da + hf * 8192, k), kIdescS, k > 0);
-                    mma_commit_warp(&bar_s_full[hf]);
+                for (int k = 0; k < D / 16; ++k)
+                    mma_bf16_ss_warp(t_dp, desc_kmajor(va, k), desc_kmajor(da + hf * 8192, k), kIdescS, k > 0);
+                mma_commit_warp(&bar_s_full[hf]);
+            };
+            // dV, dK (TS) and dQ^T (SS) of one half of pair n
+            auto issue_grads = [&](int hf, int n) {
+                const uint32_t qa = stage_q(n), da = qa + L::kTile;
+                const uint32_t t_s = tmem + 256 + hf * 128, t_dp = t_s + 64;
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16_ts_warp(t_dv, t_s + k * 8, desc_mnmajor(da, hf * 4 + k), kIdescKV,
+                                     (n > 0 || hf > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16_ts_warp(t_dk, t_dp + k * 8, desc_mnmajor(qa, hf * 4 + k), kIdescKV,
+                                     (n > 0 || hf > 0 || k > 0) ? 1u : 0u);
+                if (hf == 1) mma_commit_warp(&bar_qdo_empty[n & 1]);   // Q/dO of this stage fully read
+                const uint32_t dsa = s_base + L::kDS + hf * L::kHalfDS;
+#pragma unroll
+                for (int k = 0; k < 8; ++k) {
+                    // A = K^T (M = d): MN-major over the K tile; with d = 64 the
+                    // second 64-row atom repeats the first (those lanes are unused)
+                    const uint64_t adesc =
+                        (D == 128) ? desc_mnmajor(ka, k) : sw128_desc(ka + k * 2048, 0, 1024);
+                    mma_bf16_ss_warp(t_s, adesc, desc_mnmajor(dsa, k), kIdescQ, k > 0);
                 }
-                if (!w_ok) break;
-                // dV, dK (TS) and dQ^T (SS) of both halves
-                for (int hf = 0; hf < 2; ++hf) {
+                mma_commit_warp(&bar_dq_full[hf]);
+            };
+            // Issue order: S/dP of pair n+1, half h, goes out as soon as half h's dQ^T of
+            // pair n has been drained from TMEM, ahead of the other half's gradients, so
+            // the element-wise warps find the next scores ready when they finish pair n.
+            bool have = wait(bar_kv, 0, 33) && wait(&bar_entry[0], 0, 34);
+            have = have && ring[0].h >= 0 && wait(&bar_qdo_full[0], 0, 34);
+            if (have) {
+                tc_fence_after();
+                issue_sdp(0, 0);
+                issue_sdp(1, 0);
+            }
+            for (int n = 0; have; ++n) {
+                if (!wait(&bar_entry[(n + 1) & 3], ((n + 1) >> 2) & 1, 34)) break;
+                const bool next = ring[(n + 1) & 3].h >= 0;
+                bool w_ok = true;
+                for (int hf = 0; hf < 2 && w_ok; ++hf) {
                     if (!wait(&bar_p_ready[hf], n & 1, 36)) {
                         w_ok = false;
                         break;
                     }
                     tc_fence_after();
-                    const uint32_t t_s = tmem + 256 + hf * 128, t_dp = t_s + 64;
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        mma_bf16_ts_warp(t_dv, t_s + k * 8, desc_mnmajor(da, hf * 4 + k), kIdescKV,
-                                         (n > 0 || hf > 0 || k > 0) ? 1u : 0u);
-#pragma unroll
-                    for (int k = 0; k < 4; ++k)
-                        mma_bf16_ts_warp(t_dk, t_dp + k * 8, desc_mnmajor(qa, hf * 4 + k), kIdescKV,
-                                         (n > 0 || hf > 0 || k > 0) ? 1u : 0u);
-                    if (hf == 1) mma_commit_warp(&bar_qdo_empty[st]);   // Q/dO of this stage fully read
-                    const uint32_t dsa = s_base + L::kDS + hf * L::kHalfDS;
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        // A = K^T (M = d): MN-major over the K tile; with d = 64 the
-                        // second 64-row atom repeats the first (those lanes are unused)
-                        const uint64_t adesc =
-                            (D == 128) ? desc_mnmajor(ka, k) : sw128_desc(ka + k * 2048, 0, 1024);
-                        mma_bf16_ss_warp(t_s, adesc, desc_mnmajor(dsa, k), kIdescQ, k > 0);
+                    issue_grads(hf, n);
+                    if (!next) continue;
+                    if (!wait(&bar_dq_free[hf], n & 1, 35) ||
+                        (hf == 0 && !wait(&bar_qdo_full[(n + 1) & 1], ((n + 1) >> 1) & 1, 34))) {
+                        w_ok = false;
+                        break;
                     }
-                    mma_commit_warp(&bar_dq_full[hf]);
+                    tc_fence_after();
+                    issue_sdp(hf, n + 1);
                 }
-                if (!w_ok) break;
-                ++n;
+                if (!w_ok || !next) break;
             }
             mma_commit_warp(bar_done);
             // every MMA this warp issued must finish before TMEM is released
