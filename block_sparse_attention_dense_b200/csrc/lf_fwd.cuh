@@ -73,6 +73,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 17);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 18);
     volatile int* burst_seq = reinterpret_cast<volatile int*>(bars + 19);   // [2] bursts issued per MMA issuer
+    uint64_t* bar_p_half = bars + 20;   // [2] per query tile: P columns [0, 64) written
 
     const int h = blockIdx.y;
     const int s = blockIdx.z;
@@ -101,6 +102,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             mbar_init(&bar_v_empty[i], two ? 2 : 1);
             mbar_init(&bar_s_full[i], 1);
             mbar_init(&bar_p_ready[i], 128);
+            mbar_init(&bar_p_half[i], 128);
             mbar_init(&bar_o_done[i], 1);
         }
         mbar_init(&bar_done[0], 1);
@@ -207,14 +209,20 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 for (int j = 0; j < nk && ok; ++j) {
                     const int st = j & 1;
                     if (!wait(&bar_v_full[st], (j >> 1) & 1, 26)) break;
-                    if (!wait(&bar_p_ready[t], j & 1, 27)) break;
                     if (j + 1 < nk && !wait(&bar_k_full[(j + 1) & 1], ((j + 1) >> 1) & 1, 28)) break;
+                    if (!wait(&bar_p_half[t], j & 1, 18)) break;
                     if (!my_turn()) break;
+                    // P.V over the first 64 keys while the softmax finishes the second half
                     tc_fence_after();
                     const uint32_t va = s_base + L::kV + st * L::kTile;
 #pragma unroll
-                    for (int k = 0; k < 8; ++k)
+                    for (int k = 0; k < 4; ++k)
                         mma_bf16_ts_warp(t_o, t_s + k * 8, desc_mnmajor(va, k), kIdescO, (j > 0 || k > 0) ? 1u : 0u);
+                    if (!wait(&bar_p_ready[t], j & 1, 27)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int k = 4; k < 8; ++k)
+                        mma_bf16_ts_warp(t_o, t_s + k * 8, desc_mnmajor(va, k), kIdescO, 1u);
                     mma_commit_warp(&bar_o_done[t]);
                     mma_commit_warp(&bar_v_empty[st]);
                     if (j + 1 < nk) issue_s(j + 1);
@@ -287,6 +295,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 m_ref = mx;
                 rescale = true;
             }
+            if (__any_sync(0xffffffffu, rescale)) {
+                // O_t must hold the previous P.V product before it is rescaled (it does: S
+                // of this step completed after it); no P.V of this step has started yet
+                const bool got_o = mbar_wait_or_abort(&bar_o_done[t], (j - 1) & 1, 31, abort_flag);
+                if (!__all_sync(0xffffffffu, got_o)) { failed = true; break; }
+                tc_fence_after();
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                    float ov[32];
+                    tmem_ld32(t_o + c * 32, ov);
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) ov[e] *= alpha;
+                    tmem_st32(t_o + c * 32, ov);
+                }
+            }
             // P = 2^(scale * S - m_ref), in four chunks of 32 columns, software-pipelined:
             // the exponentials of chunk c+1 are issued ahead of the row sums, the bf16
             // packing and the TMEM store of chunk c, so that one warp keeps the MUFU busy
@@ -313,26 +336,16 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 finish(0, pa);
                 exps(2, pa);
                 finish(1, pb);
+                // the first half of P (columns [0, 64), K = 0..63 of P.V) is in TMEM
+                tmem_wait_st();
+                tc_fence_before();
+                mbar_arrive(&bar_p_half[t]);
                 exps(3, pb);
                 finish(2, pa);
                 finish(3, pb);
             }
             const float rs_all = (rs[0] + rs[1]) + (rs[2] + rs[3]);
             l_run = l_run * alpha + rs_all;
-            if (__any_sync(0xffffffffu, rescale)) {
-                // O_t must hold the previous P.V product before it is rescaled
-                const bool got_o = mbar_wait_or_abort(&bar_o_done[t], (j - 1) & 1, 31, abort_flag);
-                if (!__all_sync(0xffffffffu, got_o)) { failed = true; break; }
-                tc_fence_after();
-#pragma unroll
-                for (int c = 0; c < D / 32; ++c) {
-                    float ov[32];
-                    tmem_ld32(t_o + c * 32, ov);
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) ov[e] *= alpha;
-                    tmem_st32(t_o + c * 32, ov);
-                }
-            }
             tmem_wait_st();
             tc_fence_before();
             mbar_arrive(&bar_p_ready[t]);
