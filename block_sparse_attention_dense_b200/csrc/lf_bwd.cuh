@@ -21,8 +21,9 @@
 //   tcgen05 (SS): dQ_h^T = K_j^T dS^T_h                  (TMEM, lanes = d)
 //   dQ drain:     lane d adds column q of dQ_h^T into the fp32 accumulator;
 //                 a warp's 32 lanes hit 32 consecutive floats of one row.
-// Roles (512 threads): warp 0 TMA producer and work list, warp 1 MMA issuer (the
-// whole warp runs it, one elected lane issues), warps 4-7 element-wise half 0
+// Roles (512 threads): warp 0 TMA producer and work list, warps 1 and 2 MMA
+// issuers for query halves 0 and 1 (the whole warp runs it, one elected lane
+// issues), warps 4-7 element-wise half 0
 // (+ dV epilogue), warps 12-15 element-wise half 1 (+ dK epilogue): thread = KV
 // row = TMEM lane; warps 8-11 dQ drain (thread = head-dim index = TMEM lane).
 //
@@ -164,6 +165,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 15);
     uint64_t* bar_entry = bars + 16;      // [4] work-list ring
     PairEntry* ring = reinterpret_cast<PairEntry*>(bars + 20);   // [4] x 16 B
+    uint64_t* bar_acc0 = bars + 28;       // one phase: half 0's first dV/dK MMAs completed
 
     // KV tile fastest: CTAs resident together share one query head, so its Q,
     // dO and dQ accumulator stay in L2; the lowest tiles (most work) start first
@@ -182,13 +184,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         mbar_init(bar_kv, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&bar_qdo_full[i], 1);
-            mbar_init(&bar_qdo_empty[i], 1);
+            mbar_init(&bar_qdo_empty[i], 2);   // one commit per MMA issuer
             mbar_init(&bar_s_full[i], 1);
             mbar_init(&bar_p_ready[i], 256);
             mbar_init(&bar_dq_full[i], 1);
             mbar_init(&bar_dq_free[i], 128);
         }
-        mbar_init(bar_done, 1);
+        mbar_init(bar_done, 2);                 // one commit per MMA issuer
+        mbar_init(bar_acc0, 1);
         for (int i = 0; i < 4; ++i) mbar_init(&bar_entry[i], 1);
         *abort_flag = 0;
         fence_barrier_init();
@@ -280,10 +283,13 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             }
         }
         __syncwarp();
-    } else if (warp == 1) {
-        // ============ MMA issuer: the whole warp, one elected lane issues ============
-        // (issuing from converged code keeps the tensor pipe fed; every wait result is
-        // made warp-uniform, and each commit tracks the MMAs of the issuing lane)
+    } else if (warp == 1 || warp == 2) {
+        // ============ MMA issuers: warp 1 for query half 0, warp 2 for half 1 ============
+        // Each issuer runs its half's chain (S^T/dP^T -> element-wise -> dV, dK, dQ^T ->
+        // drain -> next S^T/dP^T) on its own, so one half's waits overlap the other
+        // half's MMAs.  The whole warp runs the code and one elected lane issues; every
+        // wait result is warp-uniform, and each commit tracks its issuing lane's MMAs.
+        const int hf = warp - 1;
         if (any) {
             auto wait = [&](uint64_t* bar, uint32_t parity, int site) {
                 return __all_sync(0xffffffffu, mbar_wait_or_abort(bar, parity, site, abort_flag));
@@ -314,7 +320,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 for (int k = 0; k < 4; ++k)
                     mma_bf16_ts_warp(t_dk, t_dp + k * 8, desc_mnmajor(qa, hf * 4 + k), kIdescKV,
                                      (n > 0 || hf > 0 || k > 0) ? 1u : 0u);
-                if (hf == 1) mma_commit_warp(&bar_qdo_empty[n & 1]);   // Q/dO of this stage fully read
+                mma_commit_warp(&bar_qdo_empty[n & 1]);   // this half is done with the Q/dO stage
                 const uint32_t dsa = s_base + L::kDS + hf * L::kHalfDS;
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
@@ -326,37 +332,30 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 }
                 mma_commit_warp(&bar_dq_full[hf]);
             };
-            // Issue order: S/dP of pair n+1, half h, goes out as soon as half h's dQ^T of
-            // pair n has been drained from TMEM, ahead of the other half's gradients, so
-            // the element-wise warps find the next scores ready when they finish pair n.
+            // Order per half: S^T/dP^T of pair n+1 goes out as soon as this half's dQ^T of
+            // pair n has been drained from TMEM.  dV and dK collect both halves in pipe
+            // order, so half 1's first gradients wait until half 0's first ones (which
+            // start the accumulators) have completed.
             bool have = wait(bar_kv, 0, 33) && wait(&bar_entry[0], 0, 34);
             have = have && ring[0].h >= 0 && wait(&bar_qdo_full[0], 0, 34);
             if (have) {
                 tc_fence_after();
-                issue_sdp(0, 0);
-                issue_sdp(1, 0);
+                issue_sdp(hf, 0);
             }
             for (int n = 0; have; ++n) {
                 if (!wait(&bar_entry[(n + 1) & 3], ((n + 1) >> 2) & 1, 34)) break;
                 const bool next = ring[(n + 1) & 3].h >= 0;
-                bool w_ok = true;
-                for (int hf = 0; hf < 2 && w_ok; ++hf) {
-                    if (!wait(&bar_p_ready[hf], n & 1, 36)) {
-                        w_ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    issue_grads(hf, n);
-                    if (!next) continue;
-                    if (!wait(&bar_dq_free[hf], n & 1, 35) ||
-                        (hf == 0 && !wait(&bar_qdo_full[(n + 1) & 1], ((n + 1) >> 1) & 1, 34))) {
-                        w_ok = false;
-                        break;
-                    }
-                    tc_fence_after();
-                    issue_sdp(hf, n + 1);
-                }
-                if (!w_ok || !next) break;
+                if (!wait(&bar_p_ready[hf], n & 1, 36)) break;
+                if (hf == 1 && n == 0 && !wait(bar_acc0, 0, 44)) break;
+                tc_fence_after();
+                issue_grads(hf, n);
+                if (hf == 0 && n == 0) mma_commit_warp(bar_acc0);
+                if (!next) break;
+                if (!wait(&bar_dq_free[hf], n & 1, 35) ||
+                    !wait(&bar_qdo_full[(n + 1) & 1], ((n + 1) >> 1) & 1, 34))
+                    break;
+                tc_fence_after();
+                issue_sdp(hf, n + 1);
             }
             mma_commit_warp(bar_done);
             // every MMA this warp issued must finish before TMEM is released
