@@ -205,7 +205,7 @@ def main():
     ap.add_argument("--rule-param", type=float, default=None)
     ap.add_argument("--seqlen", type=int, default=None, help="override the workload's length "
                     "(single-segment workloads)")
-    ap.add_argument("--cpu-prefix", type=int, default=2048,
+    ap.add_argument("--cpu-prefix", type=int, default=3072,
                     help="tokens of the oracle sample timed for cpu_baseline")
     ap.add_argument("--ref-prefix", type=int, default=1024,
                     help="tokens of the oracle sample timed per step by --impl reference")
