@@ -191,6 +191,88 @@ def config_of(w, args):
 # ---------------------------------------------------------------------------
 # LazyFlash arm
 # ---------------------------------------------------------------------------
+def run_layers(args, w):
+    """Synthetic layer-stack step: per layer a QKV projection, LazyFlash attention
+    (the autograd wrapper: exact forward, block-sparse backward), an output projection
+    and a residual add; loss <x_L, g> with a block-skewed g; backward and a plain SGD
+    update (lr 1e-9) of the random weights; every step's loss must be finite.  Timed at
+    the workload's delta against delta = 0 (the dense backward through the same
+    kernels), plus the attention's own fwd+bwd."""
+    from block_sparse_attention_dense_b200.autograd import lazyflash_attention
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    L, T, hq, hkv, d = args.layers, w.total_tokens, w.hq, w.hkv, w.d
+    inp = synthetic.make_layer_step_inputs(w, L, dev)
+    params = [p.clone().requires_grad_(True) for p in inp["wqkv"] + inp["wo"]]
+    wqkv, wo = params[:L], params[L:]
+    x0, g, cu = inp["x"], inp["g"], inp["cu_seqlens"]
+
+    def layer_step(delta):
+        x = x0
+        for l in range(L):
+            qkv = x @ wqkv[l]
+            q = qkv[:, :hq * d].reshape(T, hq, d).contiguous()
+            k = qkv[:, hq * d:(hq + hkv) * d].reshape(T, hkv, d).contiguous()
+            v = qkv[:, (hq + hkv) * d:].reshape(T, hkv, d).contiguous()
+            o = lazyflash_attention(q, k, v, cu, T, delta=delta, causal=w.causal, block_q=w.block)
+            x = x + o.reshape(T, hq * d) @ wo[l]
+        loss = (x.float() * g.float()).sum()
+        grads = torch.autograd.grad(loss, params)
+        finite.append(torch.isfinite(loss))
+        with torch.no_grad():
+            # the update runs every step; lr 1e-9 keeps the random weights (and so every
+            # later step's inputs) in range: the skewed loss gradient summed over T rows
+            # is large, and a diverging stack would time non-finite data
+            for p, gr in zip(params, grads):
+                p.sub_(gr, alpha=1e-9)
+
+    att = synthetic.make_inputs(w)
+    aq, ak, av, adout = (att[n].to(dev) for n in ("q", "k", "v", "dout"))
+    aq.requires_grad_(True)
+    ak.requires_grad_(True)
+    av.requires_grad_(True)
+
+    def attn_step(delta):
+        o = lazyflash_attention(aq, ak, av, cu, T, delta=delta, causal=w.causal, block_q=w.block)
+        torch.autograd.grad(o, (aq, ak, av), adout)
+
+    finite = []
+
+    def timed(fn, delta):
+        for _ in range(args.warmup):
+            fn(delta)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            fn(delta)
+        e1.record()
+        torch.cuda.synchronize()
+        return e0.elapsed_time(e1) / args.steps
+
+    ms = {"step": {}, "attention": {}}
+    for name, delta in (("lazyflash", w.delta), ("dense", 0.0)):
+        ms["step"][name] = timed(layer_step, delta)
+        ms["attention"][name] = timed(attn_step, delta)
+    if not bool(torch.stack(finite).all()):
+        raise SystemExit("the synthetic layer stack produced a non-finite loss")
+    line = {
+        "metric": "synthetic %d-layer step (QKV proj, LazyFlash attention, out proj, residual; "
+                  "fwd + bwd + SGD) speed-up over the dense backward (delta = 0)" % L,
+        "value": ms["step"]["dense"] / ms["step"]["lazyflash"],
+        "unit": "x",
+        "higher_is_better": True,
+        "ms_per_step": ms["step"],
+        "attention_fwd_bwd": {"ms": ms["attention"],
+                              "speedup": ms["attention"]["dense"] / ms["attention"]["lazyflash"]},
+        "steps": args.steps, "warmup": args.warmup, "n_gpus": 1,
+        "dtype": "bf16", "data": "synthetic (random weights, no data set)",
+        "config": {"workload": w.name, "layers": L, "total_tokens": T, "hq": hq, "hkv": hkv, "d": d,
+                   "hidden": hq * d, "delta": w.delta, "dO_block_scale": "LogNormal(0,%g)" % w.sigma},
+    }
+    print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -210,6 +292,8 @@ def main():
     ap.add_argument("--ref-prefix", type=int, default=1024,
                     help="tokens of the oracle sample timed per step by --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layers", type=int, default=0,
+                    help="time the synthetic layer-stack step instead (its own JSON line)")
     args = ap.parse_args()
     args.metric = "LazyFlash attn bwd ms & executed TFLOP/s at N=32K, Hq32/Hkv8 d128, delta=0.1"
     w = synthetic.WORKLOADS[args.workload]
@@ -219,6 +303,9 @@ def main():
         if w.nseq != 1:
             raise SystemExit("--seqlen applies to single-segment workloads")
         w = w.with_(seqlens=(args.seqlen,))
+    if args.layers > 0:
+        run_layers(args, w)
+        return
     rule_id = {"budget": 0, "fixed": 1, "topk": 2}[args.rule]
     rule_param = w.delta if rule_id == 0 else args.rule_param
     if rule_id != 0 and rule_param is None:

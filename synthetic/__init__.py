@@ -145,3 +145,29 @@ def random_norms(nseq: int, hq: int, nbmax: int, nb_per_seq, sigma: float, seed:
     for s, nb in enumerate(nb_per_seq):
         m[s, :, nb:] = 0.0
     return m
+
+
+def make_layer_step_inputs(w: Workload, layers: int, device, seed: int = 0) -> dict:
+    """Inputs of the synthetic layer-stack step (random weights, no data set), drawn on
+    ``device`` from a seeded torch generator: activations x [T, hq*d] ~ N(0, 1); per layer
+    W_qkv [hq*d, (hq + 2 hkv) d] and W_o [hq*d, hq*d] ~ N(0, 1/(hq*d)); and the loss
+    gradient g [T, hq*d] ~ N(0, 1) times a LogNormal(0, sigma) scale per token block,
+    shared by all heads (a per-head scale would be averaged away by the output
+    projection, which mixes the heads, before the gradient reaches the attention)."""
+    gen = torch.Generator(device=device)
+    gen.manual_seed(seed)
+    T, hidden = w.total_tokens, w.hq * w.d
+    nqkv = (w.hq + 2 * w.hkv) * w.d
+
+    def normal(shape, std):
+        return (torch.randn(shape, generator=gen, device=device, dtype=torch.float32) * std).to(torch.bfloat16)
+
+    x = normal((T, hidden), 1.0)
+    wqkv = [normal((hidden, nqkv), hidden ** -0.5) for _ in range(layers)]
+    wo = [normal((hidden, hidden), hidden ** -0.5) for _ in range(layers)]
+    g = torch.randn((T, w.hq, w.d), generator=gen, device=device, dtype=torch.float32)
+    nb = (T + w.block - 1) // w.block
+    scales = torch.empty((nb,), device=device, dtype=torch.float32).log_normal_(0.0, w.sigma, generator=gen)
+    g *= scales.repeat_interleave(w.block)[:T, None, None]
+    cu = torch.tensor([0, T], dtype=torch.int32, device=device)
+    return {"x": x, "wqkv": wqkv, "wo": wo, "g": g.reshape(T, hidden).to(torch.bfloat16), "cu_seqlens": cu}
