@@ -152,7 +152,12 @@ lf_status launch_bwd(const lf_attn_desc* d, const void* q, const void* k, const 
     float* dq_acc = reinterpret_cast<float*>(base + lay.dq);
     float* dk_acc = reinterpret_cast<float*>(base + lay.dk);
     float* dv_acc = reinterpret_cast<float*>(base + lay.dv);
-    if (cudaMemsetAsync(base, 0, lay.acc_end, st) != cudaSuccess) return LF_ERR_CUDA;
+    // dK/dV accumulators whole; the dQ accumulator only in the rows of kept blocks
+    if (cudaMemsetAsync(base + lay.dk, 0, lay.acc_end - lay.dk, st) != cudaSuccess) return LF_ERR_CUDA;
+    const dim3 blocks(nbmax_of(d), d->hq, d->nseq);
+    lf::dq_acc_zero_kept_kernel<<<blocks, 256, 0, st>>>(d->cu_seqlens, d->total_tokens, d->max_seqlen, d->hq,
+                                                        D, d->block_q, nbmax_of(d), w, dq_acc);
+    if (launch_status() != LF_OK) return LF_ERR_CUDA;
     lf::BwdParams p{};
     p.cu_seqlens = d->cu_seqlens;
     p.T = d->total_tokens;
@@ -180,12 +185,11 @@ lf_status launch_bwd(const lf_attn_desc* d, const void* q, const void* k, const 
     lf::attn_bwd_kernel<D><<<grid, lf::kBwdThreads, smem, st>>>(mq, mk, mv, mdo, p);
     if (launch_status() != LF_OK) return LF_ERR_CUDA;
     // fp32 accumulators -> bf16 results (dQ and dK take the softmax scale)
-    const size_t nq8 = (size_t)d->total_tokens * d->hq * D / 8;
     const size_t nkv8 = (size_t)d->total_tokens * d->hkv * D / 8;
-    const int bq = (int)std::min<size_t>((nq8 + 255) / 256, 148 * 16);
     const int bkv = (int)std::min<size_t>((nkv8 + 255) / 256, 148 * 16);
-    lf::acc_hmajor_to_thd_kernel<<<bq, 256, 0, st>>>(dq_acc, static_cast<uint4*>(dq),
-                                                     d->total_tokens, d->hq, D, d->softmax_scale);
+    lf::dq_acc_to_thd_kept_kernel<D><<<blocks, 256, 0, st>>>(d->cu_seqlens, d->total_tokens, d->max_seqlen,
+                                                             d->hq, d->block_q, nbmax_of(d), w, dq_acc,
+                                                             static_cast<uint4*>(dq), d->softmax_scale);
     lf::dq_convert_kernel<<<bkv, 256, 0, st>>>(reinterpret_cast<const float4*>(dk_acc),
                                                static_cast<uint4*>(dk), nkv8, d->softmax_scale);
     lf::dq_convert_kernel<<<bkv, 256, 0, st>>>(reinterpret_cast<const float4*>(dv_acc),

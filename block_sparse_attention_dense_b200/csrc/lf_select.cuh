@@ -231,7 +231,7 @@ __global__ void __launch_bounds__(32) select_kernel(
 }
 
 // ---------------------------------------------------------------------------
-// 3. dQ = scale * accumulator, rounded to bf16 (8 elements per thread).
+// 3. dK, dV = scale * accumulator, rounded to bf16 (8 elements per thread).
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) dq_convert_kernel(const float4* __restrict__ acc,
                                                          uint4* __restrict__ dq, size_t n8,
@@ -249,28 +249,54 @@ __global__ void __launch_bounds__(256) dq_convert_kernel(const float4* __restric
 }
 
 // ---------------------------------------------------------------------------
-// dQ = scale * accumulator with the head-major accumulator [H][T][D] permuted
-// to the THD output [T][H][D]; one thread converts 8 consecutive d.
+// 4. The dQ accumulator, kept blocks only.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) acc_hmajor_to_thd_kernel(const float* __restrict__ acc,
-                                                                uint4* __restrict__ out, int T,
-                                                                int H, int D, float scale) {
-    const int d8 = D / 8;
-    const size_t n8 = (size_t)T * H * d8;
-    for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n8;
-         i += (size_t)gridDim.x * blockDim.x) {
-        const int c = (int)(i % d8);
-        const size_t th = i / d8;                 // t * H + h
-        const int h = (int)(th % H);
-        const size_t t = th / H;
-        const float4* src = reinterpret_cast<const float4*>(acc + ((size_t)h * T + t) * D + c * 8);
-        const float4 a = src[0], b = src[1];
-        uint4 r;
-        r.x = pack_bf16(a.x * scale, a.y * scale);
-        r.y = pack_bf16(a.z * scale, a.w * scale);
-        r.z = pack_bf16(b.x * scale, b.y * scale);
-        r.w = pack_bf16(b.z * scale, b.w * scale);
-        out[i] = r;
+// The backward adds into the fp32 dQ accumulator only the rows of blocks whose
+// weight is non-zero (dropped blocks contribute exactly nothing), so only those rows
+// are zeroed beforehand and read afterwards; the bf16 dQ rows of the other blocks are
+// written as zeros.  One CTA per (block, head, segment); accumulator head-major
+// [H][T][D] fp32, output [T][H][D] bf16.
+__global__ void __launch_bounds__(256) dq_acc_zero_kept_kernel(const int32_t* __restrict__ cu_seqlens, int T,
+                                                               int max_seqlen, int H, int D, int block_q,
+                                                               int nbmax, const float* __restrict__ w,
+                                                               float* __restrict__ acc) {
+    const int b = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
+    int seg0, len;
+    if (!load_segment(cu_seqlens, s, T, max_seqlen, seg0, len, 50)) return;
+    if (b * block_q >= len || w[((size_t)s * H + h) * nbmax + b] == 0.f) return;
+    const int r0 = b * block_q, r1 = min(len, r0 + block_q);
+    float4* dst = reinterpret_cast<float4*>(acc + ((size_t)h * T + seg0 + r0) * D);
+    const int n4 = (r1 - r0) * D / 4;
+    for (int i = threadIdx.x; i < n4; i += blockDim.x) dst[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) dq_acc_to_thd_kept_kernel(const int32_t* __restrict__ cu_seqlens, int T,
+                                                                 int max_seqlen, int H, int block_q, int nbmax,
+                                                                 const float* __restrict__ w,
+                                                                 const float* __restrict__ acc,
+                                                                 uint4* __restrict__ out, float scale) {
+    const int b = blockIdx.x, h = blockIdx.y, s = blockIdx.z;
+    int seg0, len;
+    if (!load_segment(cu_seqlens, s, T, max_seqlen, seg0, len, 51)) return;
+    if (b * block_q >= len) return;
+    const bool kept = w[((size_t)s * H + h) * nbmax + b] != 0.f;
+    const int r0 = b * block_q, r1 = min(len, r0 + block_q);
+    constexpr int d8 = D / 8;
+    const int n = (r1 - r0) * d8;
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const int c = i % d8;
+        const size_t t = (size_t)seg0 + r0 + i / d8;
+        uint4 r = make_uint4(0u, 0u, 0u, 0u);
+        if (kept) {
+            const float4* src = reinterpret_cast<const float4*>(acc + ((size_t)h * T + t) * D + c * 8);
+            const float4 a = src[0], bb = src[1];
+            r.x = pack_bf16(a.x * scale, a.y * scale);
+            r.y = pack_bf16(a.z * scale, a.w * scale);
+            r.z = pack_bf16(bb.x * scale, bb.y * scale);
+            r.w = pack_bf16(bb.z * scale, bb.w * scale);
+        }
+        out[(t * H + h) * d8 + c] = r;
     }
 }
 
