@@ -31,6 +31,11 @@ SMALL = [
     synthetic.Workload("mha_noncausal", (300, 200), hq=2, hkv=2, d=128, block=128, sigma=1.0,
                        delta=0.05, causal=False),
     synthetic.Workload("blk64_d128", (520,), hq=4, hkv=1, d=128, block=64, sigma=2.0, delta=0.3),
+    # group of 8 query heads per KV head, d = 64 with 128-row blocks, ragged tail
+    synthetic.Workload("mqa_g8_d64", (600,), hq=8, hkv=1, d=64, block=128, sigma=1.5, delta=0.15),
+    # GQA without the causal mask, two segments, 64-row blocks
+    synthetic.Workload("gqa_noncausal", (384, 129), hq=4, hkv=2, d=64, block=64, sigma=1.5,
+                       delta=0.1, causal=False),
 ]
 
 
