@@ -448,8 +448,9 @@ def main():
                 "frac": achieved / peak, "traffic": t}
 
     roof_fwd = roof("attn_fwd_kernel", "lf_attn_fwd (one kernel)", fwd_tf)
-    roof_bwd = roof("attn_bwd_kernel", "lf_attn_bwd (memset + attn_bwd_kernel + 3 fp32->bf16 "
-                    "conversions; the kernel is ~97% of the call in the ncu launch list)", bwd_tf)
+    roof_bwd = roof("attn_bwd_kernel", "lf_attn_bwd (dK/dV memset, kept-rows dQ zeroing, "
+                    "attn_bwd_kernel, 3 fp32->bf16 conversions; the kernel is ~97% of the call in "
+                    "the ncu launch list)", bwd_tf)
     line = {
         "metric": args.metric, "value": value, "unit": "TFLOP/s", "n_gpus": n, "steps": K,
         "warmup": max(3, args.warmup), "ms_per_step": total_ms / K, "higher_is_better": True,
@@ -468,7 +469,7 @@ def main():
         "roofline_bwd": roof_bwd,
         "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / Ke, "steps": Ke},
-        "gpu_launches": 7 * K,   # fwd, norms, select, bwd, 3 accumulator conversions
+        "gpu_launches": 8 * K,   # fwd, norms, select, dQ zeroing, bwd, 3 accumulator conversions
         "clocks": clk,
     }
     if rank == 0 and n == 1 and not args.no_cpu_baseline:
