@@ -12,10 +12,13 @@
 //   softmax:  warpgroup t, thread r owns query row r (TMEM lane r): online
 //             softmax in the exp2 domain with a stale-max rule (the reference
 //             maximum moves only when the row maximum grows by more than 2^8,
-//             and only then is O rescaled in TMEM);
+//             and only then is O rescaled in TMEM); P is written in four
+//             32-column chunks, and P.V starts once the first half is stored;
 //   epilogue: O / l -> bf16, LSE = (m + log2 l) * ln 2.
-// Roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer, warps 4-7
-// softmax of tile 0, warps 8-11 softmax of tile 1.
+// Roles (384 threads): warp 0 TMA producer, warps 1 and 2 MMA issuers of tile 0
+// and tile 1 (whole warp, one elected lane issues; the two take turns so the
+// tensor pipe sees the ping-pong order), warps 4-7 softmax of tile 0, warps
+// 8-11 softmax of tile 1.
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,256+d),
 // O1 [384,384+d); P_t (bf16, packed two per column) over S_t [0,64).  Reuse
 // of a region by a later MMA relies on tcgen05.mma executing in issue order.
