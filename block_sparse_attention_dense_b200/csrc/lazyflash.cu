@@ -118,6 +118,15 @@ lf_status launch_fwd(const lf_attn_desc* d, const void* q, const void* k, const 
     if (cudaFuncSetAttribute(lf::attn_fwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem) != cudaSuccess)
         return LF_ERR_CUDA;
+    // The kernel's warpgroups resize their register budgets (setmaxnreg); the larger
+    // budget can only be granted from the registers the block was launched with, so a
+    // build that launches with fewer than the budgets add up to must not run (its
+    // softmax warps would wait for registers that never come).
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, lf::attn_fwd_kernel<D>) != cudaSuccess) return LF_ERR_CUDA;
+    const int launch_regs = (fa.numRegs + 7) / 8 * 8;
+    if (launch_regs * lf::kFwdThreads < 128 * lf::kFwdCtrlRegs + 256 * lf::kFwdSoftmaxRegs)
+        return LF_ERR_UNSUPPORTED;
     // one CTA per pair of query tiles; pair index fastest so that the CTAs resident
     // together share a head (its K/V stay in L2)
     dim3 grid((ntiles_of(d) + 1) / 2, d->hq, d->nseq);
