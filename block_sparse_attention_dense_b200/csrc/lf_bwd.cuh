@@ -150,7 +150,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     using L = BwdSmem<D>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    float* lse2_s = reinterpret_cast<float*>(smem + L::kVec);
+    float* lse2_s = reinterpret_cast<float*>(smem + L::kVec);   // -LSE * log2(e) per column
     float* dvec_s = lse2_s + 128;
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBars);
     uint64_t* bar_kv = bars + 0;
@@ -392,7 +392,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     l2 = prm.lse[idx] * 1.4426950408889634f;
                     dd = prm.Dvec[idx];
                 }
-                lse2_s[col] = l2;
+                lse2_s[col] = -l2;   // stored negated: the exponent is one packed FMA
                 dvec_s[col] = dd;
             }
             named_bar_sync(2, 256);
@@ -426,15 +426,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         const int col0 = hf * 64 + c * 16 + 4 * e4;
                         const float4 l4 = *reinterpret_cast<const float4*>(lse2_s + col0);
                         const float4 d4 = *reinterpret_cast<const float4*>(dvec_s + col0);
-                        const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-                        const float dv_[4] = {d4.x, d4.y, d4.z, d4.w};
+                        const float2 sc2 = make_float2(prm.scale_log2, prm.scale_log2);
+                        const float2 w2 = make_float2(w, w);
                         float pw[4], dsw[4];
+                        // two columns per packed instruction
 #pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            float p = fast_exp2(fmaf(__uint_as_float(sr[4 * e4 + u]), prm.scale_log2, -lv[u]));
-                            if (diag && kv_local > q0 + col0 + u) p = 0.f;
-                            pw[u] = p * w;
-                            dsw[u] = pw[u] * (__uint_as_float(dr[4 * e4 + u]) - dv_[u]);
+                        for (int u = 0; u < 4; u += 2) {
+                            const float2 nl = u ? make_float2(l4.z, l4.w) : make_float2(l4.x, l4.y);
+                            const float2 dv2 = u ? make_float2(d4.z, d4.w) : make_float2(d4.x, d4.y);
+                            const float2 s2 = make_float2(__uint_as_float(sr[4 * e4 + u]),
+                                                          __uint_as_float(sr[4 * e4 + u + 1]));
+                            const float2 dp2 = make_float2(__uint_as_float(dr[4 * e4 + u]),
+                                                           __uint_as_float(dr[4 * e4 + u + 1]));
+                            const float2 x = f2_fma(s2, sc2, nl);
+                            float p0 = fast_exp2(x.x), p1 = fast_exp2(x.y);
+                            if (diag && kv_local > q0 + col0 + u) p0 = 0.f;
+                            if (diag && kv_local > q0 + col0 + u + 1) p1 = 0.f;
+                            const float2 pw2 = f2_mul(make_float2(p0, p1), w2);
+                            const float2 ds2 = f2_mul(pw2, f2_sub(dp2, dv2));
+                            pw[u] = pw2.x;
+                            pw[u + 1] = pw2.y;
+                            dsw[u] = ds2.x;
+                            dsw[u + 1] = ds2.y;
                         }
                         pk[2 * e4] = pack_bf16(pw[0], pw[1]);
                         pk[2 * e4 + 1] = pack_bf16(pw[2], pw[3]);

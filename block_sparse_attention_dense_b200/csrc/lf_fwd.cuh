@@ -317,17 +317,26 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
             // the exponentials of chunk c+1 are issued ahead of the row sums, the bf16
             // packing and the TMEM store of chunk c, so that one warp keeps the MUFU busy
             const float neg_m = -m_ref;
-            float rs[4] = {0.f, 0.f, 0.f, 0.f};
+            // (scale and subtract, and the row sums, in packed pairs)
+            const float2 sc2 = make_float2(prm.scale_log2, prm.scale_log2);
+            const float2 nm2 = make_float2(neg_m, neg_m);
             auto exps = [&](int c, float (&p)[32]) {
 #pragma unroll
-                for (int e = 0; e < 32; ++e) p[e] = fast_exp2(fmaf(sv[c * 32 + e], prm.scale_log2, neg_m));
+                for (int e = 0; e < 32; e += 2) {
+                    const float2 x = f2_fma(make_float2(sv[c * 32 + e], sv[c * 32 + e + 1]), sc2, nm2);
+                    p[e] = fast_exp2(x.x);
+                    p[e + 1] = fast_exp2(x.y);
+                }
             };
+            float2 rsA = make_float2(0.f, 0.f), rsB = make_float2(0.f, 0.f);
             auto finish = [&](int c, const float (&p)[32]) {
                 uint32_t pk[16];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
-                    rs[(e & 1) * 2] += p[2 * e];
-                    rs[(e & 1) * 2 + 1] += p[2 * e + 1];
+                    if (e & 1)
+                        rsB = f2_add(rsB, make_float2(p[2 * e], p[2 * e + 1]));
+                    else
+                        rsA = f2_add(rsA, make_float2(p[2 * e], p[2 * e + 1]));
                     pk[e] = pack_bf16(p[2 * e], p[2 * e + 1]);
                 }
                 tmem_st16(t_s + c * 16, pk);   // P (packed) over S columns already read
@@ -347,7 +356,7 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
                 finish(2, pa);
                 finish(3, pb);
             }
-            const float rs_all = (rs[0] + rs[1]) + (rs[2] + rs[3]);
+            const float rs_all = (rsA.x + rsA.y) + (rsB.x + rsB.y);
             l_run = l_run * alpha + rs_all;
             tmem_wait_st();
             tc_fence_before();
