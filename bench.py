@@ -149,6 +149,22 @@ def oracle_sample(w: synthetic.Workload, inp, prefix: int, seed=0, step=0):
     return dt, f + b, threads
 
 
+def max_over_ranks(values, dist=None, device=None):
+    """Element-wise maximum of every rank's `values` (the job is as slow as its slowest
+    rank); a single process returns them unchanged."""
+    if dist is None:
+        return [float(v) for v in values]
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t]
+
+
+def whole_job_tflops(n_ranks, steps, flops_per_step, ms):
+    """Throughput of the whole job: each of `n_ranks` ranks ran `steps` steps of
+    `flops_per_step` (weak scaling) within `ms`, the maximum over ranks."""
+    return n_ranks * steps * flops_per_step / (ms * 1e-3) / 1e12
+
+
 def run_reference(args, w, rank):
     if rank != 0:
         return
@@ -417,15 +433,12 @@ def main():
     e2e_ms = e2s.elapsed_time(e2e)
 
     # ---- max over ranks
-    if dist is not None:
-        tt = torch.tensor([total_ms, e2e_ms], device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        total_ms, e2e_ms = float(tt[0]), float(tt[1])
+    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dist, dev)
 
     n = world
     step_fl = fwd_fl + bwd_exec_fl
-    value = n * K * step_fl / (total_ms * 1e-3) / 1e12
-    e2e_val = n * Ke * step_fl / (e2e_ms * 1e-3) / 1e12
+    value = whole_job_tflops(n, K, step_fl, total_ms)
+    e2e_val = whole_job_tflops(n, Ke, step_fl, e2e_ms)
     peaks = _load_json(os.path.join(ROOT, "MEASURED_PEAKS.json"))
     if peaks:
         peak, peak_src = float(peaks["bf16_tflops_sustained"]), "measured (sustained)"
