@@ -77,7 +77,66 @@ _CLOCK_FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.
                  "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
 
-class ClockSampler:
+_REASON_NAMES = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+                 ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+                 ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+                 ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
+
+
+def _summarise(sm, mx, reasons, source):
+    return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+            "reasons": sorted(reasons), "samples": len(sm), "source": source}
+
+
+class _NvmlSampler:
+    """SM clock and clock-event reasons every 5 ms from a thread of this process
+    (read-only NVML queries), so that even a short timed region is covered."""
+
+    def __init__(self, device_index: int):
+        import threading
+        import pynvml
+        self.nv = pynvml
+        pynvml.nvmlInit()
+        uuid = str(torch.cuda.get_device_properties(device_index).uuid)
+        if not uuid.startswith("GPU-"):
+            uuid = "GPU-" + uuid
+        self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid.encode() if isinstance(uuid, str) else uuid)
+        self.mx = float(pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM))
+        self.bits = [(name, getattr(pynvml, attr)) for name, attr in _REASON_NAMES]
+        self.sm, self.reasons = [], set()
+        self.stop_ev = threading.Event()
+        self.t = threading.Thread(target=self._run, daemon=True)
+        self.t.start()
+        t0 = time.time()
+        while not self.sm and time.time() - t0 < 2.0:   # first sample before timing starts
+            time.sleep(0.001)
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop_ev.is_set():
+            try:
+                self.sm.append(float(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.bits:
+                    if bits & bit:
+                        self.reasons.add(name)
+            except Exception:
+                return
+            self.stop_ev.wait(0.005)
+
+    def stop(self):
+        self.stop_ev.set()
+        self.t.join(timeout=5)
+        try:
+            self.nv.nvmlShutdown()
+        except Exception:
+            pass
+        return _summarise(self.sm, self.mx, self.reasons, "nvml, 5 ms")
+
+
+class _SmiSampler:
+    """Fallback: nvidia-smi in a subprocess (first sample after ~0.1-0.5 s)."""
+
     def __init__(self, device_index: int):
         self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
         uuid = None
@@ -121,8 +180,15 @@ class ClockSampler:
             for n, v in zip(names, r[5:9]):
                 if v.lower() == "active":
                     reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        return _summarise(sm, mx, reasons, "nvidia-smi, 100 ms")
+
+
+def ClockSampler(device_index: int):
+    """Starts sampling now; .stop() returns the summary for the JSON line."""
+    try:
+        return _NvmlSampler(device_index)
+    except Exception:
+        return _SmiSampler(device_index)
 
 
 # ---------------------------------------------------------------------------
