@@ -92,6 +92,21 @@ bool make_thd_map(CUtensorMap* m, const void* base, int T, int H, int D) {
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// [T][H][d] fp32 accumulator -> 3-D map (d, H, T), 32 x 1 x 128 boxes (128 bytes of a
+// row each), 128-byte swizzle: the layout the backward stages its dK/dV tiles in.
+bool make_acc_map(CUtensorMap* m, float* base, int T, int H, int D) {
+    EncodeTiledFn enc = encode_tiled();
+    if (!enc) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 4, (cuuint64_t)H * D * 4};
+    const cuuint32_t box[3] = {32, 1, 128};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, base, dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 inline lf_status launch_status() {
     return cudaGetLastError() == cudaSuccess ? LF_OK : LF_ERR_CUDA;
 }
@@ -161,6 +176,10 @@ lf_status launch_bwd(const lf_attn_desc* d, const void* q, const void* k, const 
     float* dq_acc = reinterpret_cast<float*>(base + lay.dq);
     float* dk_acc = reinterpret_cast<float*>(base + lay.dk);
     float* dv_acc = reinterpret_cast<float*>(base + lay.dv);
+    CUtensorMap mdvacc, mdkacc;
+    if (!make_acc_map(&mdvacc, dv_acc, d->total_tokens, d->hkv, D) ||
+        !make_acc_map(&mdkacc, dk_acc, d->total_tokens, d->hkv, D))
+        return LF_ERR_CUDA;
     // dK/dV accumulators whole; the dQ accumulator only in the rows of kept blocks
     if (cudaMemsetAsync(base + lay.dk, 0, lay.acc_end - lay.dk, st) != cudaSuccess) return LF_ERR_CUDA;
     const dim3 blocks(nbmax_of(d), d->hq, d->nseq);
@@ -184,14 +203,12 @@ lf_status launch_bwd(const lf_attn_desc* d, const void* q, const void* k, const 
     p.kept_idx = kidx;
     p.kept_cnt = kcnt;
     p.dq_acc = dq_acc;
-    p.dk_acc = dk_acc;
-    p.dv_acc = dv_acc;
     const uint32_t smem = lf::BwdSmem<D>::kAlloc;
     if (cudaFuncSetAttribute(lf::attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem) != cudaSuccess)
         return LF_ERR_CUDA;
     dim3 grid(ntiles_of(d), d->hq, d->nseq);
-    lf::attn_bwd_kernel<D><<<grid, lf::kBwdThreads, smem, st>>>(mq, mk, mv, mdo, p);
+    lf::attn_bwd_kernel<D><<<grid, lf::kBwdThreads, smem, st>>>(mq, mk, mv, mdo, mdvacc, mdkacc, p);
     if (launch_status() != LF_OK) return LF_ERR_CUDA;
     // fp32 accumulators -> bf16 results (dQ and dK take the softmax scale)
     const size_t nkv8 = (size_t)d->total_tokens * d->hkv * D / 8;

@@ -47,9 +47,11 @@ struct BwdParams {
     const int32_t* kept_idx;   // [nseq][hq][nbmax]
     const int32_t* kept_cnt;   // [nseq][hq]
     float* dq_acc;             // [hq][T][D] fp32 (head-major), zeroed by the caller
-    float* dk_acc;             // [T][hkv][D] fp32 (unscaled), zeroed by the caller
-    float* dv_acc;             // [T][hkv][D] fp32, zeroed by the caller
+    // dK (unscaled) and dV go to [T][hkv][D] fp32 accumulators, zeroed by the caller,
+    // through the tensor maps the kernel is given (32 x 1 x 128 boxes, 128-byte swizzle)
 };
+
+constexpr uint32_t kAccBox = 128 * 32 * 4;   // one staged 32-column fp32 box of a KV tile
 
 template <int D>
 struct BwdSmem {
@@ -146,8 +148,10 @@ template <int D>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const __grid_constant__ CUtensorMap tm_dvacc, const __grid_constant__ CUtensorMap tm_dkacc,
                     BwdParams prm) {
     using L = BwdSmem<D>;
+    static_assert(2 * (D / 32) * kAccBox <= 4 * L::kTile, "dK/dV staging must fit the Q/dO buffers");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     float* lse2_s = reinterpret_cast<float*>(smem + L::kVec);   // -LSE * log2(e) per column
@@ -199,6 +203,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         prefetch_tensormap(&tm_k);
         prefetch_tensormap(&tm_v);
         prefetch_tensormap(&tm_do);
+        prefetch_tensormap(&tm_dvacc);
+        prefetch_tensormap(&tm_dkacc);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, 512);
@@ -369,6 +375,10 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const int kv_local = jt * 128 + r;
         const bool kv_valid = kv_local < len;
+        // P = 0 where kv_cmp > the query's index: the key follows the query (causal), or
+        // the KV row lies past the segment's end (its key belongs to the next segment, so
+        // its exponent is not bounded by this query's LSE and must not reach the products)
+        const int kv_cmp = !kv_valid ? 0x7fffffff : (prm.causal ? kv_local : (int)0x80000000);
         int n = 0;
         bool more = any, failed = false;
         for (;;) {
@@ -396,9 +406,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 dvec_s[col] = dd;
             }
             named_bar_sync(2, 256);
-            const bool diag = prm.causal && qt == jt;
             for (int hf = 0; hf < 2; ++hf) {
-                const float w = kv_valid ? (hf ? e.w1 : e.w0) : 0.f;
+                const float w = hf ? e.w1 : e.w0;
                 const uint32_t t_s = tmem + 256 + hf * 128 + lane_off, t_dp = t_s + 64;
                 const uint32_t dsa = s_base + L::kDS + hf * L::kHalfDS;
                 const bool got = mbar_wait_or_abort(&bar_s_full[hf], n & 1, 38, abort_flag);
@@ -440,8 +449,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                                                            __uint_as_float(dr[4 * e4 + u + 1]));
                             const float2 x = f2_fma(s2, sc2, nl);
                             float p0 = fast_exp2(x.x), p1 = fast_exp2(x.y);
-                            if (diag && kv_local > q0 + col0 + u) p0 = 0.f;
-                            if (diag && kv_local > q0 + col0 + u + 1) p1 = 0.f;
+                            if (kv_cmp > q0 + col0 + u) p0 = 0.f;
+                            if (kv_cmp > q0 + col0 + u + 1) p1 = 0.f;
                             const float2 pw2 = f2_mul(make_float2(p0, p1), w2);
                             const float2 ds2 = f2_mul(pw2, f2_sub(dp2, dv2));
                             pw[u] = pw2.x;
@@ -469,24 +478,38 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             if (!failed) ++n;
         }
         // ---- epilogue: warpgroup 0 adds dV, warpgroup 1 adds dK (unscaled) into the
-        // fp32 accumulators of the KV head (the GQA sum over query heads) ----
+        // fp32 accumulators of the KV head (the GQA sum over query heads).  Each thread
+        // stages its KV row in the Q/dO buffers, free once every MMA has completed, as
+        // 32-column boxes with the 128-byte swizzle; one thread then adds the boxes with
+        // TMA reduce-adds (rows past the segment's end hold exact zeros: P and dS are
+        // 0 there; rows past the tensor's end are clipped by the copy) ----
         bool have = n > 0 && !failed && !*abort_flag;
-        if (have) have = mbar_wait_or_abort(bar_done, 0, 39, abort_flag);
-        have = __all_sync(0xffffffffu, have);
+        if (have) have = mbar_wait_or_abort(bar_done, 0, 39, abort_flag) && !*abort_flag;
+        // one decision per warpgroup: all 128 threads meet at the staging barrier
+        have = !named_bar_or(6 + wg, 128, !have);
         if (have) {
             tc_fence_after();
-            float* dst = (hf_epi ? prm.dk_acc : prm.dv_acc) + ((size_t)(kv_row0 + r) * prm.hkv + g) * D;
             const uint32_t t_acc = (hf_epi ? t_dk : t_dv) + lane_off;
+            uint8_t* stage = smem + L::kQdo + hf_epi * (D / 32) * kAccBox;
 #pragma unroll 1
             for (int c = 0; c < D / 32; ++c) {
                 float v[32];
                 tmem_ld32(t_acc + c * 32, v);
-                if (kv_valid) {
+                const uint32_t row = smem_addr(stage + c * kAccBox) + r * 128;
 #pragma unroll
-                    for (int e4 = 0; e4 < 8; ++e4)
-                        atomicAdd(reinterpret_cast<float4*>(dst + c * 32 + 4 * e4),
-                                  make_float4(v[4 * e4], v[4 * e4 + 1], v[4 * e4 + 2], v[4 * e4 + 3]));
-                }
+                for (int k = 0; k < 8; ++k)
+                    st_shared_v4(row + ((k ^ (r & 7)) << 4), __float_as_uint(v[4 * k]),
+                                 __float_as_uint(v[4 * k + 1]), __float_as_uint(v[4 * k + 2]),
+                                 __float_as_uint(v[4 * k + 3]));
+            }
+            fence_proxy_async_smem();
+            named_bar_sync(6 + wg, 128);
+            if (r == 0) {
+                const CUtensorMap* map = hf_epi ? &tm_dkacc : &tm_dvacc;
+                for (int c = 0; c < D / 32; ++c)
+                    tma_reduce_add_3d(map, stage + c * kAccBox, 32 * c, g, kv_row0);
+                bulk_commit_group();
+                bulk_wait0();   // added (and the staging read) before the CTA exits
             }
         }
     } else if (warp >= 8 && warp < 12) {

@@ -171,6 +171,36 @@ def test_heavy_budget_leaves_unreached_kv_tiles_zero():
             assert torch.all(bufs.dv[j * 128:(j + 1) * 128] == 0)
 
 
+@pytest.mark.parametrize("block", [64, 128])
+def test_noncausal_keys_of_the_next_segment_stay_out(block):
+    """Without the causal mask, the last KV tile of a segment also holds the next
+    segment's keys.  Here half of those keys share a large first coordinate with
+    this segment's queries, so their scores (about 450) lie far above this segment's
+    LSE and exp() of them overflows fp32; they must contribute nothing (the
+    article's attention is per sequence: a key of another segment has P = 0)."""
+    w = synthetic.Workload("segment_edge", (200, 150), hq=2, hkv=1, d=64, block=block, sigma=1.0,
+                           delta=0.0, causal=False)
+    inp = synthetic.make_inputs(w)
+    q, k = inp["q"].clone(), inp["k"].clone()
+    # segment 0's queries against segment 1's keys: +-60 * 60 / sqrt(64) = +-450 (the
+    # sign alternates so that no coordinate of segment 1's keys is a common offset,
+    # which would leave dQ's bf16 rounding noise on a sum that is exactly zero)
+    q[:200, :, 0] = 60.0
+    k[200:, :, 0] = torch.tensor([60.0, -60.0]).repeat(75)[:, None].to(k.dtype)
+    k[:200, :, 0] = 0.0      # the scores within each segment stay ordinary
+    q[200:, :, 0] = 0.0
+    inp = dict(inp, q=q, k=k)
+    desc, dev, bufs = run_step(w, inp)
+    cu = w.cu_seqlens()
+    o_ref, lse_ref = oracle.attn_fwd(cu, inp["q"], inp["k"], inp["v"], w.scale, w.causal)
+    assert np.abs(_cpu(bufs.o) - o_ref).max() < O_TOL
+    dq_ref, dk_ref, dv_ref = oracle.attn_bwd(cu, inp["q"], inp["k"], inp["v"], inp["dout"],
+                                             w.scale, w.block, None, w.causal)
+    for got, ref in ((bufs.dq, dq_ref), (bufs.dk, dk_ref), (bufs.dv, dv_ref)):
+        assert torch.isfinite(got).all()
+        assert rel_fro(_cpu(got), ref) < GRAD_TOL
+
+
 def test_same_seed_step_reproduces_and_steps_differ():
     w = synthetic.GQA_MID.with_(seqlens=(2048,))
     inp = synthetic.make_inputs(w)
