@@ -78,6 +78,26 @@ struct PairEntry {
     float w0, w1;   // block weights of the tile's two 64-row halves
 };
 
+// First index i in list[0, cnt) with list[i] >= key (the list ascends), found by
+// the whole warp: each round probes 32 evenly spaced entries at once and keeps the
+// bracket between the last one below the key and the first one at or above it, so
+// a list of up to 1024 entries takes two rounds of loads instead of ten dependent
+// ones.  Every lane must call it and gets the same answer.
+__device__ __forceinline__ int lower_bound_warp(const int32_t* list, int cnt, int key) {
+    const int lane = threadIdx.x & 31;
+    int lo = 0, hi = cnt;
+    while (lo < hi) {
+        const int step = (hi - lo + 31) >> 5;
+        const int i = lo + lane * step;
+        const unsigned below = __ballot_sync(0xffffffffu, i < hi && list[i] < key);
+        const int nb = __popc(below);     // the probes below the key form a prefix
+        const int new_hi = min(hi, lo + nb * step);
+        lo = nb == 0 ? lo : lo + (nb - 1) * step + 1;
+        hi = nb == 0 ? lo : new_hi;
+    }
+    return lo;
+}
+
 // Walks the kept query tiles of heads g*G .. g*G+G-1 of one segment in
 // ascending order of (head, tile) (the backward uses G = 1: one head).
 struct KeptTileWalk {
@@ -100,24 +120,32 @@ struct KeptTileWalk {
         first_block = p.causal ? (jt * 128) / p.block_q : 0;
         nb = (len + p.block_q - 1) / p.block_q;
     }
-    __device__ void open_head() {
+    // `warp`: the whole warp calls this, converged (the search is shared)
+    __device__ void open_head(bool warp) {
         h = g * G + hh;
         const size_t base = ((size_t)s * hq + h) * nbmax;
         list = kept_idx + base;
         cnt = min(max(kept_cnt[(size_t)s * hq + h], 0), nbmax);
         // first kept block >= first_block (lists are ascending)
-        int lo = 0, hi = cnt;
-        while (lo < hi) {
-            const int mid = (lo + hi) >> 1;
-            if (list[mid] < first_block) lo = mid + 1; else hi = mid;
+        if (first_block == 0) {
+            pos = 0;
+        } else if (warp) {
+            pos = lower_bound_warp(list, cnt, first_block);
+        } else {
+            int lo = 0, hi = cnt;
+            while (lo < hi) {
+                const int mid = (lo + hi) >> 1;
+                if (list[mid] < first_block) lo = mid + 1; else hi = mid;
+            }
+            pos = lo;
         }
-        pos = lo;
     }
-    // Moves to the next tile; returns false when the walk is over.
+    // Moves to the next tile; returns false when the walk is over.  The first call
+    // is made by whole warps (converged); later calls by any single thread.
     __device__ bool next(bool first) {
         if (first) {
             hh = 0;
-            open_head();
+            open_head(true);
         } else {
             // skip the other blocks of the tile just processed
             while (pos < cnt && (list[pos] * block_q) / 128 == tile) ++pos;
@@ -125,7 +153,7 @@ struct KeptTileWalk {
         for (;;) {
             while (pos >= cnt) {
                 if (++hh >= G) return false;
-                open_head();
+                open_head(false);
             }
             const int b = list[pos];
             if (b >= 0 && b < nb) {
