@@ -113,6 +113,42 @@ def test_selection_bit_exact_given_norms(case, delta):
         np.testing.assert_array_equal(kidx.cpu().numpy(), ref["kept_idx"])
 
 
+def test_selection_at_the_largest_block_count():
+    """The selection holds one segment's norms in shared memory as fp64 (200 KB):
+    25,600 blocks is the largest count it takes, bit-exact there; one block more
+    is refused before any launch."""
+    nbig = 200 * 1024 // 8
+    w = synthetic.Workload("sel_max", (nbig * 128,), hq=1, hkv=1, d=64, block=128, sigma=2.0,
+                           delta=0.1)
+    nb = nb_per_seq(w)
+    m = synthetic.random_norms(1, 1, w.nbmax, nb, 2.0, seed=11)
+    cu = torch.as_tensor(w.cu_seqlens()).cuda()
+    desc = desc_for(w, cu)
+    dummy = torch.zeros(w.total_tokens, 1, 64, dtype=torch.bfloat16, device="cuda")
+    norm = torch.as_tensor(m, device="cuda")
+    D = torch.empty(1, w.total_tokens, device="cuda")
+    tau = torch.empty(1, 1, dtype=torch.float64, device="cuda")
+    wt = torch.empty(1, 1, w.nbmax, device="cuda")
+    keep = torch.empty(1, 1, w.nbmax, dtype=torch.uint8, device="cuda")
+    kidx = torch.empty(1, 1, w.nbmax, dtype=torch.int32, device="cuda")
+    kcnt = torch.empty(1, 1, dtype=torch.int32, device="cuda")
+    lf.lf_block_select(desc, dummy, dummy, w.delta, 5, 6, lf.LF_SELECT_NORMS_GIVEN, norm, D, tau, wt,
+                       keep, kidx, kcnt)
+    lf.lf_check_device_error()
+    ref = oracle.select(m, nb, w.delta, 5, 6)
+    np.testing.assert_array_equal(tau.cpu().numpy().view(np.uint64), ref["tau"].view(np.uint64))
+    np.testing.assert_array_equal(keep.cpu().numpy(), ref["keep"])
+    np.testing.assert_array_equal(wt.cpu().numpy().view(np.uint32), ref["w"].view(np.uint32))
+    np.testing.assert_array_equal(kcnt.cpu().numpy(), ref["kept_cnt"])
+    np.testing.assert_array_equal(kidx.cpu().numpy(), ref["kept_idx"])
+    w2 = w.with_(seqlens=(nbig * 128 + 1,))
+    cu2 = torch.as_tensor(w2.cu_seqlens()).cuda()
+    with pytest.raises(lf.LfError) as err:
+        lf.lf_block_select(desc_for(w2, cu2), dummy, dummy, w.delta, 5, 6, lf.LF_SELECT_NORMS_GIVEN,
+                           norm, D, tau, wt, keep, kidx, kcnt)
+    assert err.value.code == lf.LF_ERR_UNSUPPORTED
+
+
 @pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
 def test_backward_matches_oracle(w):
     inp = synthetic.make_inputs(w)
@@ -229,7 +265,13 @@ def test_empty_batch_is_a_noop():
 # Full-size workloads, in the launch configuration the bench times: outputs the
 # oracle can compute one by one (sampled rows) plus properties at any size.
 # ---------------------------------------------------------------------------
-@pytest.mark.parametrize("w", [synthetic.HEADLINE, synthetic.VARLEN], ids=lambda w: w.name)
+# one 256K-token segment with d = 64 and 64-row blocks: 4096 blocks per head in the
+# selection and in the backward's kept lists
+LONG_D64 = synthetic.Workload("long_d64", (262144,), hq=2, hkv=1, d=64, block=64, sigma=2.0,
+                              delta=0.1)
+
+
+@pytest.mark.parametrize("w", [synthetic.HEADLINE, synthetic.VARLEN, LONG_D64], ids=lambda w: w.name)
 def test_full_size_sampled_parity(w):
     inp = synthetic.make_inputs(w)
     desc, dev, bufs = run_step(w, inp)
