@@ -142,9 +142,9 @@ lf_status launch_fwd(const lf_attn_desc* d, const void* q, const void* k, const 
     const int launch_regs = (fa.numRegs + 7) / 8 * 8;
     if (launch_regs * lf::kFwdThreads < 128 * lf::kFwdCtrlRegs + 256 * lf::kFwdSoftmaxRegs)
         return LF_ERR_UNSUPPORTED;
-    // one CTA per pair of query tiles; pair index fastest so that the CTAs resident
-    // together share a head (its K/V stay in L2)
-    dim3 grid((ntiles_of(d) + 1) / 2, d->hq, d->nseq);
+    // one CTA per pair of query tiles; the query heads of one KV head together, their
+    // longest pairs first (x = pair rank * group + head in group, y = KV head)
+    dim3 grid(((ntiles_of(d) + 1) / 2) * (d->hq / d->hkv), d->hkv, d->nseq);
     lf::attn_fwd_kernel<D><<<grid, lf::kFwdThreads, smem, st>>>(mq, mk, mv, p);
     return launch_status();
 }
