@@ -195,6 +195,9 @@ lf_status launch_bwd(const lf_attn_desc* d, const void* q, const void* k, const 
     p.block_q = d->block_q;
     p.nbmax = nbmax_of(d);
     p.max_seqlen = d->max_seqlen;
+    // two query heads of one KV head per CTA where the group allows it: half the CTAs,
+    // so half the per-CTA start and finish; both heads' Q, dO and dQ stay in L2
+    p.heads_per_cta = (d->hq / d->hkv) % 2 == 0 ? 2 : 1;
     p.scale = d->softmax_scale;
     p.scale_log2 = d->softmax_scale * 1.4426950408889634f;
     p.lse = lse;
@@ -207,7 +210,7 @@ lf_status launch_bwd(const lf_attn_desc* d, const void* q, const void* k, const 
     if (cudaFuncSetAttribute(lf::attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              smem) != cudaSuccess)
         return LF_ERR_CUDA;
-    dim3 grid(ntiles_of(d), d->hq, d->nseq);
+    dim3 grid(ntiles_of(d), d->hq / p.heads_per_cta, d->nseq);
     lf::attn_bwd_kernel<D><<<grid, lf::kBwdThreads, smem, st>>>(mq, mk, mv, mdo, mdvacc, mdkacc, p);
     if (launch_status() != LF_OK) return LF_ERR_CUDA;
     // fp32 accumulators -> bf16 results (dQ and dK take the softmax scale)

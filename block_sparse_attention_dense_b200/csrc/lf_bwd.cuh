@@ -4,13 +4,15 @@
 // only kept query blocks are loaded and computed, and their output gradient
 // carries the weight 1/p).
 //
-// One CTA owns a 128-row KV tile j of one segment for ONE query head h and
-// walks the kept query tiles t of h (t >= j when causal) from the compacted
-// kept-block list.  CTAs are ordered KV tile fastest, so the CTAs resident at
-// any time share one head: that head's Q, dO and fp32 dQ accumulator stay in
-// L2, where the dQ reductions run at L2 rather than HBM speed.  The GQA sum over
-// the heads of a KV head is done by fp32 reductions of each CTA's dK/dV tile
-// (one per CTA, not per pair).  Each 128-row query tile is handled as two
+// One CTA owns a 128-row KV tile j of one segment for one or two query heads of
+// the same KV head and walks their kept query tiles t (t >= j when causal) from
+// the compacted kept-block lists.  CTAs are ordered KV tile fastest, so the CTAs
+// resident at any time share those heads: their Q, dO and fp32 dQ accumulators
+// (64 MB at 32K tokens) stay in L2, where the dQ reductions run at L2 rather
+// than HBM speed.  The GQA sum over the heads of a KV head runs in TMEM for the
+// CTA's own heads and by TMA reduce-adds of each CTA's dK/dV tile into fp32
+// accumulators across CTAs (one per CTA, not per pair).  Each 128-row query tile
+// is handled as two
 // 64-column halves, one per element-wise warpgroup, so that the element-wise
 // work on one half overlaps the tensor-core work on the other.  Per half:
 //   tcgen05 (SS): S^T  = K_j Q_h^T,  dP^T = V_j dO_h^T        (TMEM, fp32)
@@ -39,6 +41,7 @@ namespace lf {
 struct BwdParams {
     const int32_t* cu_seqlens;
     int T, hq, hkv, causal, block_q, nbmax, max_seqlen;
+    int heads_per_cta;         // 1 or 2 query heads of one KV head per CTA
     float scale;               // softmax_scale
     float scale_log2;          // softmax_scale * log2(e)
     const float* lse;          // [hq][T], natural log
@@ -98,19 +101,20 @@ __device__ __forceinline__ int lower_bound_warp(const int32_t* list, int cnt, in
     return lo;
 }
 
-// Walks the kept query tiles of heads g*G .. g*G+G-1 of one segment in
-// ascending order of (head, tile) (the backward uses G = 1: one head).
+// Walks the kept query tiles of heads g*G .. g*G+G-1 (G <= 2) of one segment in
+// ascending order of (head, tile).  init() is called by whole warps, converged: it
+// finds every head's first kept block >= first_block with the warp-parallel search,
+// so that later steps (by any single thread) only read the lists forward.
 struct KeptTileWalk {
     const int32_t* kept_idx;
-    const int32_t* kept_cnt;
     int nbmax, hq, G, g, s, block_q, first_block, nb;
     int hh, pos, cnt;
+    int start0, start1, cnt0, cnt1;   // per head of the group
     const int32_t* list;
     int tile, h;
 
     __device__ void init(const BwdParams& p, int G_, int g_, int s_, int jt, int len) {
         kept_idx = p.kept_idx;
-        kept_cnt = p.kept_cnt;
         nbmax = p.nbmax;
         hq = p.hq;
         G = G_;
@@ -119,33 +123,26 @@ struct KeptTileWalk {
         block_q = p.block_q;
         first_block = p.causal ? (jt * 128) / p.block_q : 0;
         nb = (len + p.block_q - 1) / p.block_q;
-    }
-    // `warp`: the whole warp calls this, converged (the search is shared)
-    __device__ void open_head(bool warp) {
-        h = g * G + hh;
-        const size_t base = ((size_t)s * hq + h) * nbmax;
-        list = kept_idx + base;
-        cnt = min(max(kept_cnt[(size_t)s * hq + h], 0), nbmax);
-        // first kept block >= first_block (lists are ascending)
-        if (first_block == 0) {
-            pos = 0;
-        } else if (warp) {
-            pos = lower_bound_warp(list, cnt, first_block);
-        } else {
-            int lo = 0, hi = cnt;
-            while (lo < hi) {
-                const int mid = (lo + hi) >> 1;
-                if (list[mid] < first_block) lo = mid + 1; else hi = mid;
-            }
-            pos = lo;
+        start1 = cnt1 = 0;
+        for (int i = 0; i < G; ++i) {
+            const int hi = g * G + i;
+            const int32_t* l = kept_idx + ((size_t)s * hq + hi) * nbmax;
+            const int c = min(max(p.kept_cnt[(size_t)s * hq + hi], 0), nbmax);
+            const int st = first_block == 0 ? 0 : lower_bound_warp(l, c, first_block);
+            if (i == 0) { start0 = st; cnt0 = c; } else { start1 = st; cnt1 = c; }
         }
     }
-    // Moves to the next tile; returns false when the walk is over.  The first call
-    // is made by whole warps (converged); later calls by any single thread.
+    __device__ void open_head() {
+        h = g * G + hh;
+        list = kept_idx + ((size_t)s * hq + h) * nbmax;
+        cnt = hh == 0 ? cnt0 : cnt1;
+        pos = hh == 0 ? start0 : start1;
+    }
+    // Moves to the next tile; returns false when the walk is over.
     __device__ bool next(bool first) {
         if (first) {
             hh = 0;
-            open_head(true);
+            open_head();
         } else {
             // skip the other blocks of the tile just processed
             while (pos < cnt && (list[pos] * block_q) / 128 == tile) ++pos;
@@ -153,7 +150,7 @@ struct KeptTileWalk {
         for (;;) {
             while (pos >= cnt) {
                 if (++hh >= G) return false;
-                open_head(false);
+                open_head();
             }
             const int b = list[pos];
             if (b >= 0 && b < nb) {
@@ -202,12 +199,12 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     // KV tile fastest: CTAs resident together share one query head, so its Q,
     // dO and dQ accumulator stay in L2; the lowest tiles (most work) start first
     const int jt = blockIdx.x;
-    const int hq_ = blockIdx.y;             // query head
+    const int hgrp = blockIdx.y;            // query heads hgrp*G .. hgrp*G+G-1, G = heads_per_cta
     const int s = blockIdx.z;
     int seg0, len;
     if (!load_segment(prm.cu_seqlens, s, prm.T, prm.max_seqlen, seg0, len, 30)) return;
     if (jt * 128 >= len) return;
-    const int g = hq_ / (prm.hq / prm.hkv); // its KV head
+    const int g = hgrp * prm.heads_per_cta / (prm.hq / prm.hkv);   // their KV head
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const uint32_t s_base = smem_addr(smem);
@@ -248,7 +245,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
 
     // Does this KV tile have any work?  (every role sees the same answer)
     KeptTileWalk walk;
-    walk.init(prm, 1, hq_, s, jt, len);
+    walk.init(prm, prm.heads_per_cta, hgrp, s, jt, len);
     const bool any = walk.next(true);
 
     constexpr uint32_t kIdescS = idesc_bf16(128, 64, 0, 0);    // S^T, dP^T halves
