@@ -180,8 +180,23 @@ lf_status launch_bwd(const lf_attn_desc* d, const void* q, const void* k, const 
     if (!make_acc_map(&mdvacc, dv_acc, d->total_tokens, d->hkv, D) ||
         !make_acc_map(&mdkacc, dk_acc, d->total_tokens, d->hkv, D))
         return LF_ERR_CUDA;
-    // dK/dV accumulators whole; the dQ accumulator only in the rows of kept blocks
-    if (cudaMemsetAsync(base + lay.dk, 0, lay.acc_end - lay.dk, st) != cudaSuccess) return LF_ERR_CUDA;
+    // up to four query heads of one KV head per CTA (half or a quarter of the CTAs pay
+    // the start and finish); with the whole group in one CTA, dK/dV are final in TMEM
+    // and go straight to the bf16 outputs, otherwise through fp32 accumulators
+    const int group = d->hq / d->hkv;
+    const int heads_per_cta = group % 4 == 0 ? 4 : group % 2 == 0 ? 2 : 1;
+    const bool kv_direct = heads_per_cta == group;
+    // the outputs (direct) or the dK/dV accumulators zeroed whole: rows no CTA writes
+    // (no kept block reaches them, or outside every segment) read as 0; the dQ
+    // accumulator is zeroed only in the rows of kept blocks
+    const size_t nkv = (size_t)d->total_tokens * d->hkv * D;
+    if (kv_direct) {
+        if (cudaMemsetAsync(dk, 0, nkv * 2, st) != cudaSuccess ||
+            cudaMemsetAsync(dv, 0, nkv * 2, st) != cudaSuccess)
+            return LF_ERR_CUDA;
+    } else if (cudaMemsetAsync(base + lay.dk, 0, lay.acc_end - lay.dk, st) != cudaSuccess) {
+        return LF_ERR_CUDA;
+    }
     const dim3 blocks(nbmax_of(d), d->hq, d->nseq);
     lf::dq_acc_zero_kept_kernel<<<blocks, 256, 0, st>>>(d->cu_seqlens, d->total_tokens, d->max_seqlen, d->hq,
                                                         D, d->block_q, nbmax_of(d), w, dq_acc);
@@ -195,9 +210,10 @@ lf_status launch_bwd(const lf_attn_desc* d, const void* q, const void* k, const 
     p.block_q = d->block_q;
     p.nbmax = nbmax_of(d);
     p.max_seqlen = d->max_seqlen;
-    // two query heads of one KV head per CTA where the group allows it: half the CTAs,
-    // so half the per-CTA start and finish; both heads' Q, dO and dQ stay in L2
-    p.heads_per_cta = (d->hq / d->hkv) % 2 == 0 ? 2 : 1;
+    p.heads_per_cta = heads_per_cta;
+    p.kv_out_direct = kv_direct ? 1 : 0;
+    p.dk_out = static_cast<__nv_bfloat16*>(dk);
+    p.dv_out = static_cast<__nv_bfloat16*>(dv);
     p.scale = d->softmax_scale;
     p.scale_log2 = d->softmax_scale * 1.4426950408889634f;
     p.lse = lse;
@@ -219,10 +235,12 @@ lf_status launch_bwd(const lf_attn_desc* d, const void* q, const void* k, const 
     lf::dq_acc_to_thd_kept_kernel<D><<<blocks, 256, 0, st>>>(d->cu_seqlens, d->total_tokens, d->max_seqlen,
                                                              d->hq, d->block_q, nbmax_of(d), w, dq_acc,
                                                              static_cast<uint4*>(dq), d->softmax_scale);
-    lf::dq_convert_kernel<<<bkv, 256, 0, st>>>(reinterpret_cast<const float4*>(dk_acc),
-                                               static_cast<uint4*>(dk), nkv8, d->softmax_scale);
-    lf::dq_convert_kernel<<<bkv, 256, 0, st>>>(reinterpret_cast<const float4*>(dv_acc),
-                                               static_cast<uint4*>(dv), nkv8, 1.0f);
+    if (!kv_direct) {
+        lf::dq_convert_kernel<<<bkv, 256, 0, st>>>(reinterpret_cast<const float4*>(dk_acc),
+                                                   static_cast<uint4*>(dk), nkv8, d->softmax_scale);
+        lf::dq_convert_kernel<<<bkv, 256, 0, st>>>(reinterpret_cast<const float4*>(dv_acc),
+                                                   static_cast<uint4*>(dv), nkv8, 1.0f);
+    }
     return launch_status();
 }
 

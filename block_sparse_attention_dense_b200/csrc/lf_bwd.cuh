@@ -51,7 +51,12 @@ struct BwdParams {
     const int32_t* kept_cnt;   // [nseq][hq]
     float* dq_acc;             // [hq][T][D] fp32 (head-major), zeroed by the caller
     // dK (unscaled) and dV go to [T][hkv][D] fp32 accumulators, zeroed by the caller,
-    // through the tensor maps the kernel is given (32 x 1 x 128 boxes, 128-byte swizzle)
+    // through the tensor maps the kernel is given (32 x 1 x 128 boxes, 128-byte swizzle);
+    // when a CTA covers the whole query group of its KV head (kv_out_direct) they go
+    // instead, final, to the bf16 outputs [T][hkv][D], zeroed by the caller
+    int kv_out_direct;
+    __nv_bfloat16* dk_out;
+    __nv_bfloat16* dv_out;
 };
 
 constexpr uint32_t kAccBox = 128 * 32 * 4;   // one staged 32-column fp32 box of a KV tile
@@ -101,7 +106,7 @@ __device__ __forceinline__ int lower_bound_warp(const int32_t* list, int cnt, in
     return lo;
 }
 
-// Walks the kept query tiles of heads g*G .. g*G+G-1 (G <= 2) of one segment in
+// Walks the kept query tiles of heads g*G .. g*G+G-1 (G <= 4) of one segment in
 // ascending order of (head, tile).  init() is called by whole warps, converged: it
 // finds every head's first kept block >= first_block with the warp-parallel search,
 // so that later steps (by any single thread) only read the lists forward.
@@ -109,7 +114,7 @@ struct KeptTileWalk {
     const int32_t* kept_idx;
     int nbmax, hq, G, g, s, block_q, first_block, nb;
     int hh, pos, cnt;
-    int start0, start1, cnt0, cnt1;   // per head of the group
+    int starts[4], cnts[4];           // per head of the group
     const int32_t* list;
     int tile, h;
 
@@ -123,20 +128,27 @@ struct KeptTileWalk {
         block_q = p.block_q;
         first_block = p.causal ? (jt * 128) / p.block_q : 0;
         nb = (len + p.block_q - 1) / p.block_q;
-        start1 = cnt1 = 0;
-        for (int i = 0; i < G; ++i) {
-            const int hi = g * G + i;
-            const int32_t* l = kept_idx + ((size_t)s * hq + hi) * nbmax;
-            const int c = min(max(p.kept_cnt[(size_t)s * hq + hi], 0), nbmax);
-            const int st = first_block == 0 ? 0 : lower_bound_warp(l, c, first_block);
-            if (i == 0) { start0 = st; cnt0 = c; } else { start1 = st; cnt1 = c; }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            starts[i] = cnts[i] = 0;
+            if (i < G) {
+                const int hi = g * G + i;
+                const int32_t* l = kept_idx + ((size_t)s * hq + hi) * nbmax;
+                const int c = min(max(p.kept_cnt[(size_t)s * hq + hi], 0), nbmax);
+                cnts[i] = c;
+                starts[i] = first_block == 0 ? 0 : lower_bound_warp(l, c, first_block);
+            }
         }
     }
     __device__ void open_head() {
         h = g * G + hh;
         list = kept_idx + ((size_t)s * hq + h) * nbmax;
-        cnt = hh == 0 ? cnt0 : cnt1;
-        pos = hh == 0 ? start0 : start1;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+            if (i == hh) {
+                cnt = cnts[i];
+                pos = starts[i];
+            }
     }
     // Moves to the next tile; returns false when the walk is over.
     __device__ bool next(bool first) {
@@ -512,7 +524,29 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         if (have) have = mbar_wait_or_abort(bar_done, 0, 39, abort_flag) && !*abort_flag;
         // one decision per warpgroup: all 128 threads meet at the staging barrier
         have = !named_bar_or(6 + wg, 128, !have);
-        if (have) {
+        if (have && prm.kv_out_direct) {
+            // the CTA holds its KV head's whole query group: the tile is final, so it
+            // goes straight to the bf16 output (dK takes the softmax scale); rows past
+            // the segment's end belong to the next segment and are not written
+            tc_fence_after();
+            const uint32_t t_acc = (hf_epi ? t_dk : t_dv) + lane_off;
+            const float sc = hf_epi ? prm.scale : 1.f;
+            __nv_bfloat16* dst = (hf_epi ? prm.dk_out : prm.dv_out) + ((size_t)(kv_row0 + r) * prm.hkv + g) * D;
+#pragma unroll 1
+            for (int c = 0; c < D / 32; ++c) {
+                float v[32];
+                tmem_ld32(t_acc + c * 32, v);
+                uint32_t pk[16];
+#pragma unroll
+                for (int k = 0; k < 16; ++k) pk[k] = pack_bf16(v[2 * k] * sc, v[2 * k + 1] * sc);
+                if (kv_valid) {
+                    uint4* o = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        o[k] = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
+                }
+            }
+        } else if (have) {
             tc_fence_after();
             const uint32_t t_acc = (hf_epi ? t_dk : t_dv) + lane_off;
             uint8_t* stage = smem + L::kQdo + hf_epi * (D / 32) * kAccBox;
