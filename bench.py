@@ -196,6 +196,14 @@ def ClockSampler(device_index: int):
 # ---------------------------------------------------------------------------
 # CPU oracle sample (the cpu_baseline and the reference arm)
 # ---------------------------------------------------------------------------
+def kernels_per_step(w: synthetic.Workload) -> int:
+    """This library's kernels in one step: forward; norms and selection; dQ
+    zeroing, backward and dQ conversion; plus the dK/dV conversions when the
+    backward's CTAs cannot hold a whole query group (group size not 1, 2 or 4)."""
+    group = w.hq // w.hkv
+    return 6 + (0 if group in (1, 2, 4) else 2)
+
+
 def oracle_sample(w: synthetic.Workload, inp, prefix: int, seed=0, step=0):
     """The oracle's forward, selection and weighted backward on the first
     `prefix` tokens of segment 0 (a causal prefix is itself a complete problem),
@@ -590,7 +598,7 @@ def main():
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / Ke, "steps": Ke,
                 "copies": "pinned host buffers; uploads and downloads on two side streams, "
                           "device inputs and outputs double-buffered"},
-        "gpu_launches": 8 * K,   # fwd, norms, select, dQ zeroing, bwd, 3 accumulator conversions
+        "gpu_launches": kernels_per_step(w) * K,
         "clocks": clk,
     }
     if rank == 0 and n == 1 and not args.no_cpu_baseline:
