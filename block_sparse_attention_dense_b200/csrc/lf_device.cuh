@@ -144,18 +144,10 @@ __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulate.
-__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
-// Warp-wide forms of the MMA issue and commit: the whole warp executes them and one
+// D[tmem] (+)= A * B^T, bf16 inputs, fp32 accumulate: A from shared memory (the _ss
+// form) or from tensor memory (the _ts form: M x K bf16 packed two per 32-bit column,
+// row m in lane m), B from shared memory.
+// The MMA issue and commit are warp-wide: the whole warp executes them and one
 // elected lane issues.  Issuing from converged code keeps the descriptors warp-uniform,
 // which roughly halves the time a warp needs to issue one MMA (a single-lane issue costs
 // about as long as a 128x128x16 MMA takes to run, so the tensor pipe would starve).
@@ -185,14 +177,6 @@ __device__ __forceinline__ void mma_commit_warp(uint64_t* bar) {
         "{\n\t.reg .pred e;\n\t.reg .b32 r;\n\t"
         "elect.sync r|e, 0xffffffff;\n\t"
         "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];\n\t}" ::"r"(
-            smem_addr(bar))
-        : "memory");
-}
-
-// Arrive once on `bar` when every MMA this thread issued so far has completed.
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
             smem_addr(bar))
         : "memory");
 }
@@ -343,18 +327,6 @@ __device__ __forceinline__ float fmax3(float a, float b, float c) {
 
 namespace lf {
 
-// D[tmem] (+)= A[tmem] * B[smem]^T: A (M x K, bf16 packed two per 32-bit
-// column, row m in lane m) read from tensor memory.
-__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-        "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
 // 16 consecutive 32-bit columns of this thread's TMEM lane (raw bits).
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&v)[16]) {
     asm volatile(
@@ -451,7 +423,7 @@ __device__ __forceinline__ void tmem_wait_ld_regs(uint32_t (&a)[16], uint32_t (&
 }
 
 // Element-wise add of a shared-memory box into global memory through TMA
-// (no multicast).  The source must not be modified until bulk_wait_read0().
+// (no multicast).  The source must not be modified until bulk_wait0().
 __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, const void* src, int x,
                                                   int y, int z) {
     asm volatile(
@@ -463,11 +435,8 @@ __device__ __forceinline__ void tma_reduce_add_3d(const CUtensorMap* map, const 
 __device__ __forceinline__ void bulk_commit_group() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
-// All bulk copies this thread committed have finished reading shared memory.
-__device__ __forceinline__ void bulk_wait_read0() {
-    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-}
-// ... and have completed (their global writes are performed).
+// Every bulk copy this thread committed has completed (its global writes are performed,
+// its shared-memory source read).
 __device__ __forceinline__ void bulk_wait0() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
