@@ -176,8 +176,9 @@ lf_status lf_attn_bwd(const lf_attn_desc* desc, const void* q, const void* k, co
  *   The first call on a device looks up the array's device address
  *   (cudaGetSymbolAddress, with that device current); make that first call
  *   before any stream capture.  The call never calls cudaMalloc, cudaFree or an
- *   allocating library routine; the accumulators are cleared at the start of
- *   every call.
+ *   allocating library routine; the accumulators a call uses are cleared at
+ *   its start (dK and dV need none when the query heads of each KV head fit
+ *   in one CTA, i.e. hq/hkv is 1, 2 or 4: they are then written directly).
  *   All calls on a device share the one array and it keeps the last call's
  *   contents: calls that may overlap on the GPU (different streams, or host
  *   threads without ordering) race on it and produce wrong dQ. */
