@@ -4,17 +4,18 @@
 // only kept query blocks are loaded and computed, and their output gradient
 // carries the weight 1/p).
 //
-// One CTA owns a 128-row KV tile j of one segment for one or two query heads of
-// the same KV head and walks their kept query tiles t (t >= j when causal) from
-// the compacted kept-block lists.  CTAs are ordered KV tile fastest, so the CTAs
-// resident at any time share those heads: their Q, dO and fp32 dQ accumulators
-// (64 MB at 32K tokens) stay in L2, where the dQ reductions run at L2 rather
-// than HBM speed.  The GQA sum over the heads of a KV head runs in TMEM for the
-// CTA's own heads and by TMA reduce-adds of each CTA's dK/dV tile into fp32
-// accumulators across CTAs (one per CTA, not per pair).  Each 128-row query tile
-// is handled as two
-// 64-column halves, one per element-wise warpgroup, so that the element-wise
-// work on one half overlaps the tensor-core work on the other.  Per half:
+// One CTA owns a 128-row KV tile j of one segment for up to four query heads of
+// the same KV head (the whole query group when it has 1, 2 or 4 heads) and walks
+// their kept query tiles t (t >= j when causal) from the compacted kept-block
+// lists, head by head.  CTAs are ordered KV tile fastest, so the CTAs resident at
+// any time share those heads: their Q, dO and fp32 dQ accumulators (about 128 MB
+// for four heads at 32K tokens) stay largely in L2, where the dQ reductions run at
+// L2 rather than HBM speed.  dK/dV sum the CTA's heads in TMEM; when the CTA holds
+// the whole query group they are final and stored as bf16, otherwise each CTA's
+// tile is added into fp32 accumulators by TMA reduce-adds (one per CTA, not per
+// pair).  Each 128-row query tile is handled as two 64-column halves, so that the
+// element-wise work on one half overlaps the tensor-core work on the other.
+// Per half:
 //   tcgen05 (SS): S^T  = K_j Q_h^T,  dP^T = V_j dO_h^T        (TMEM, fp32)
 //   element-wise: P = exp2(S*scale*log2e - LSE*log2e), dS = P (dP - D), both
 //                 times the block weight; P^T and dS^T rounded to bf16 back
@@ -25,9 +26,9 @@
 //                 a warp's 32 lanes hit 32 consecutive floats of one row.
 // Roles (512 threads): warp 0 TMA producer and work list, warps 1 and 2 MMA
 // issuers for query halves 0 and 1 (the whole warp runs it, one elected lane
-// issues), warps 4-7 element-wise half 0
-// (+ dV epilogue), warps 12-15 element-wise half 1 (+ dK epilogue): thread = KV
-// row = TMEM lane; warps 8-11 dQ drain (thread = head-dim index = TMEM lane).
+// issues), warps 4-7 and 12-15 element-wise on columns [0, 32) and [32, 64) of
+// each half (+ the dV and the dK epilogue respectively): thread = KV row = TMEM
+// lane; warps 8-11 dQ drain (thread = head-dim index = TMEM lane).
 //
 // Tensor memory (512 columns): dV [0,128) dK [128,256); half 0: S^T/P^T/dQ^T
 // [256,320), dP^T/dS^T [320,384); half 1: [384,448), [448,512).  Reuse of a
@@ -41,7 +42,7 @@ namespace lf {
 struct BwdParams {
     const int32_t* cu_seqlens;
     int T, hq, hkv, causal, block_q, nbmax, max_seqlen;
-    int heads_per_cta;         // 1 or 2 query heads of one KV head per CTA
+    int heads_per_cta;         // 1, 2 or 4 query heads of one KV head per CTA
     float scale;               // softmax_scale
     float scale_log2;          // softmax_scale * log2(e)
     const float* lse;          // [hq][T], natural log
