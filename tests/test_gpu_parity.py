@@ -36,6 +36,10 @@ SMALL = [
     # GQA without the causal mask, two segments, 64-row blocks
     synthetic.Workload("gqa_noncausal", (384, 129), hq=4, hkv=2, d=64, block=64, sigma=1.5,
                        delta=0.1, causal=False),
+    # three query heads per KV head: one head per backward CTA, dK/dV through the fp32
+    # accumulators; the forward's head-in-group index with an odd group
+    synthetic.Workload("gqa3_d128", (333, 200), hq=6, hkv=2, d=128, block=128, sigma=1.5,
+                       delta=0.1),
 ]
 
 
