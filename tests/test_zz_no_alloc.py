@@ -19,9 +19,12 @@ from _helpers import rel_fro, run_step
 GRAD_TOL = 1e-2   # the backward parity tolerance of the other GPU tests
 
 
+# two query heads per KV head: dK/dV written directly by whole-group CTAs; three: dK/dV
+# through the fp32 accumulators in the static array
 @pytest.mark.gpu
-def test_static_scratch_backward_matches_workspace_backward_twice():
-    w = synthetic.Workload("no_alloc", (700, 300), hq=4, hkv=2, d=128, block=128, sigma=1.5,
+@pytest.mark.parametrize("hq", [4, 6], ids=["group2_direct", "group3_accumulators"])
+def test_static_scratch_backward_matches_workspace_backward_twice(hq):
+    w = synthetic.Workload("no_alloc", (700, 300), hq=hq, hkv=2, d=128, block=128, sigma=1.5,
                            delta=0.1)
     # one full step through the ordinary entry points (caller workspace)
     desc, dev, bufs = run_step(w, synthetic.make_inputs(w), seed=2, step=3)
