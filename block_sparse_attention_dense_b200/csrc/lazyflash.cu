@@ -126,6 +126,7 @@ lf_status launch_fwd(const lf_attn_desc* d, const void* q, const void* k, const 
     p.hkv = d->hkv;
     p.causal = d->causal;
     p.max_seqlen = d->max_seqlen;
+    p.nseq = d->nseq;
     p.scale_log2 = d->softmax_scale * 1.4426950408889634f;
     p.o = static_cast<__nv_bfloat16*>(o);
     p.lse = lse;
@@ -144,7 +145,9 @@ lf_status launch_fwd(const lf_attn_desc* d, const void* q, const void* k, const 
         return LF_ERR_UNSUPPORTED;
     // one CTA per pair of query tiles; the query heads of one KV head together, their
     // longest pairs first (x = pair rank * group + head in group, y = KV head)
-    dim3 grid(((ntiles_of(d) + 1) / 2) * (d->hq / d->hkv), d->hkv, d->nseq);
+    // (x: pairs of query tiles over all segments, flattened; see segment_of_unit)
+    const long long pair_units = ((long long)d->total_tokens + 255ll * d->nseq) >> 8;
+    dim3 grid(static_cast<unsigned>(pair_units * (d->hq / d->hkv)), d->hkv, 1);
     lf::attn_fwd_kernel<D><<<grid, lf::kFwdThreads, smem, st>>>(mq, mk, mv, p);
     return launch_status();
 }

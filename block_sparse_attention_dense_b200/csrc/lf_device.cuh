@@ -42,6 +42,32 @@ __device__ __forceinline__ bool load_segment(const int32_t* cu, int s, int T, in
     return true;
 }
 
+// Flattened grids over variable-length segments: segment s's work units (tiles of
+// 2^u rows) start at F(s) = (cu[s] + (2^u - 1) s) >> u.  F(s+1) - F(s) is at least
+// ceil(len_s / 2^u) and at most one more, so a grid of (T + (2^u - 1) nseq) >> u units
+// covers every segment with at most one idle unit each.  Returns the segment of unit
+// x (the last s with F(s) <= x), or -1; the whole warp calls it, converged, and probes
+// 32 segment starts per round.
+__device__ __forceinline__ int segment_of_unit(const int32_t* cu, int nseq, int x, int u) {
+    const int lane = threadIdx.x & 31;
+    int lo = 0, hi = nseq;   // the first s with F(s) > x lies in [lo, hi]
+    while (lo < hi) {
+        const int step = (hi - lo + 31) >> 5;
+        const int i = lo + lane * step;
+        const bool le =
+            i < hi && ((static_cast<long long>(cu[i]) + ((1ll << u) - 1) * i) >> u) <= x;
+        const unsigned below = __ballot_sync(0xffffffffu, le);
+        const int nb = __popc(below);   // F ascends: the probes at or below x form a prefix
+        const int new_hi = min(hi, lo + nb * step);
+        lo = nb == 0 ? lo : lo + (nb - 1) * step + 1;
+        hi = nb == 0 ? lo : new_hi;
+    }
+    return lo - 1;
+}
+__device__ __forceinline__ int first_unit_of_segment(int seg0, int s, int u) {
+    return static_cast<int>((static_cast<long long>(seg0) + ((1ll << u) - 1) * s) >> u);
+}
+
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }

@@ -32,7 +32,7 @@ namespace lf {
 
 struct FwdParams {
     const int32_t* cu_seqlens;
-    int T, hq, hkv, causal, max_seqlen;
+    int T, hq, hkv, causal, max_seqlen, nseq;
     float scale_log2;          // softmax_scale * log2(e)
     __nv_bfloat16* o;
     float* lse;
@@ -78,18 +78,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     volatile int* burst_seq = reinterpret_cast<volatile int*>(bars + 19);   // [2] bursts issued per MMA issuer
     uint64_t* bar_p_half = bars + 20;   // [2] per query tile: P columns [0, 64) written
 
-    // blockIdx.x = pair rank * G + query head within the KV head's group, blockIdx.y =
-    // KV head: the G query heads that share a KV head run together, longest rows
-    // first, so their K/V stay in L2 and each group's work outlasts its heaviest CTA
+    // blockIdx.x = pair * G + query head within the KV head's group, the pairs of
+    // 256 query rows running over all segments, segment by segment; blockIdx.y = KV
+    // head.  The G query heads that share a KV head run together, longest rows first,
+    // so their K/V stay in L2 and each group's work outlasts its heaviest CTA.
     const int G = prm.hq / prm.hkv;
     const int g = blockIdx.y;
     const int h = g * G + static_cast<int>(blockIdx.x) % G;
-    const int s = blockIdx.z;
+    const int pg = static_cast<int>(blockIdx.x) / G;
+    const int s = segment_of_unit(prm.cu_seqlens, prm.nseq, pg, 8);
+    if (s < 0) return;
     int seg0, len;
     if (!load_segment(prm.cu_seqlens, s, prm.T, prm.max_seqlen, seg0, len, 20)) return;
     const int ntiles = (len + 127) >> 7;
     const int npairs = (ntiles + 1) >> 1;
-    const int m = npairs - 1 - static_cast<int>(blockIdx.x) / G;   // longest rows first
+    const int m = npairs - 1 - (pg - first_unit_of_segment(seg0, s, 8));   // longest rows first
     if (m < 0) return;
     const bool two = 2 * m + 1 < ntiles;                     // tile 1 exists
     // KV tiles each query tile needs
