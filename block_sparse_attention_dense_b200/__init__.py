@@ -5,7 +5,8 @@ liblazyflash.so.  PyTorch provides device memory and streams.  There is no CPU
 fallback: importing the binding without the built library raises.
 
 Functions keep the C names: lf_attn_fwd, lf_block_select, lf_attn_bwd,
-lf_workspace_size, lf_check_device_error, lf_status_string.  Tensors are torch
+lf_workspace_size, lf_sync_status (alias lf_check_device_error),
+lf_status_string.  Tensors are torch
 CUDA tensors in the layouts the header states; the stream defaults to torch's
 current stream.
 """
@@ -25,7 +26,7 @@ LF_SELECT_NORMS_GIVEN = 0x1
 LF_RULE_BUDGET, LF_RULE_FIXED_FRACTION, LF_RULE_TOPK = 0, 1, 2
 
 EXPORTED = ("lf_workspace_size", "lf_attn_fwd", "lf_block_select", "lf_attn_bwd",
-            "lf_check_device_error", "lf_status_string")
+            "lf_sync_status", "lf_check_device_error", "lf_status_string")
 
 
 class LfError(RuntimeError):
@@ -76,6 +77,8 @@ def _load():
     L.lf_attn_bwd.restype = i32
     L.lf_check_device_error.argtypes = [vp]
     L.lf_check_device_error.restype = i32
+    L.lf_sync_status.argtypes = [vp]
+    L.lf_sync_status.restype = i32
     _lib = L
     return L
 
@@ -174,21 +177,28 @@ def lf_watchdog_selftest(limit_log2=24, stream=None):
     _check(L.lf_watchdog_selftest(int(limit_log2), _stream(stream)), "lf_watchdog_selftest")
 
 
+def lf_sync_status(stream=None):
+    """Synchronizes the stream; raises LfError for a device-side failure of an
+    earlier call (and clears it)."""
+    _check(_load().lf_sync_status(_stream(stream)), "lf_sync_status")
+
+
 def lf_check_device_error(stream=None):
     _check(_load().lf_check_device_error(_stream(stream)), "lf_check_device_error")
 
 
 class Buffers:
     """Device buffers of one attention layer for one LazyFlash step (torch
-    allocations: plumbing only)."""
+    allocations: plumbing only).  With forward=False the forward's outputs (o, lse)
+    are not allocated: the caller already holds them."""
 
-    def __init__(self, desc: lf_attn_desc, device="cuda"):
+    def __init__(self, desc: lf_attn_desc, device="cuda", forward: bool = True):
         T, hq, hkv, d = desc.total_tokens, desc.hq, desc.hkv, desc.d
         nbmax = (desc.max_seqlen + desc.block_q - 1) // desc.block_q
         bf = dict(dtype=torch.bfloat16, device=device)
         f32 = dict(dtype=torch.float32, device=device)
-        self.o = torch.empty(T, hq, d, **bf)
-        self.lse = torch.empty(hq, T, **f32)
+        self.o = torch.empty(T, hq, d, **bf) if forward else None
+        self.lse = torch.empty(hq, T, **f32) if forward else None
         self.norm = torch.empty(desc.nseq, hq, nbmax, **f32)
         self.D = torch.empty(hq, T, **f32)
         self.tau = torch.empty(desc.nseq, hq, dtype=torch.float64, device=device)

@@ -26,7 +26,7 @@ _step_counter = itertools.count()
 class LazyFlashAttention(torch.autograd.Function):
     @staticmethod
     def forward(ctx, q, k, v, cu_seqlens, max_seqlen, delta, seed, step, causal, block_q,
-                softmax_scale):
+                softmax_scale, selection_out):
         for t in (q, k, v):
             if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
                 raise ValueError("q, k, v must be contiguous bf16 CUDA tensors")
@@ -42,6 +42,7 @@ class LazyFlashAttention(torch.autograd.Function):
         ctx.delta = float(delta)
         ctx.seed = int(seed)
         ctx.step = int(next(_step_counter) if step is None else step)
+        ctx.selection_out = selection_out
         return o
 
     @staticmethod
@@ -49,20 +50,26 @@ class LazyFlashAttention(torch.autograd.Function):
         q, k, v, o, lse, cu_seqlens = ctx.saved_tensors
         desc = ctx.desc
         dout = grad_o.to(torch.bfloat16).contiguous()
-        bufs = Buffers(desc, device=q.device)
+        # the backward's own buffers only: o and lse are the forward's saved tensors
+        bufs = Buffers(desc, device=q.device, forward=False)
         lf_block_select(desc, dout, o, ctx.delta, ctx.seed, ctx.step, 0, bufs.norm, bufs.D,
                         bufs.tau, bufs.w, bufs.keep, bufs.kept_idx, bufs.kept_cnt)
         lf_attn_bwd(desc, q, k, v, o, lse, dout, bufs.D, bufs.w, bufs.kept_idx, bufs.kept_cnt,
                     bufs.dq, bufs.dk, bufs.dv, bufs.ws)
-        ctx.selection = {"tau": bufs.tau, "keep": bufs.keep, "weight": bufs.w}
-        return bufs.dq, bufs.dk, bufs.dv, None, None, None, None, None, None, None, None
+        if ctx.selection_out is not None:
+            ctx.selection_out.update(norm=bufs.norm, tau=bufs.tau, keep=bufs.keep,
+                                     weight=bufs.w, kept_cnt=bufs.kept_cnt, step=ctx.step)
+        return bufs.dq, bufs.dk, bufs.dv, None, None, None, None, None, None, None, None, None
 
 
 def lazyflash_attention(q, k, v, cu_seqlens, max_seqlen, delta=0.1, seed=0, step=None,
-                        causal=True, block_q=128, softmax_scale=None):
+                        causal=True, block_q=128, softmax_scale=None, selection_out=None):
     """Dense attention forward, LazyFlash block-sparse backward.
 
     ``step`` defaults to a process-wide counter, so every backward draws a
-    fresh mask; pass it explicitly to replay a draw."""
+    fresh mask; pass it explicitly to replay a draw.  If ``selection_out`` is a
+    dict, the backward stores in it the selection it drew: block norms ``norm``,
+    thresholds ``tau``, ``keep``, block weights ``weight`` ([nseq, hq, nbmax]
+    device tensors), ``kept_cnt`` and the Philox ``step`` used."""
     return LazyFlashAttention.apply(q, k, v, cu_seqlens, max_seqlen, delta, seed, step, causal,
-                                    block_q, softmax_scale)
+                                    block_q, softmax_scale, selection_out)

@@ -291,6 +291,50 @@ lf_status static_ws_address(void** out) {
     return LF_OK;
 }
 
+// Device-side errors (an expired bounded wait, a bad segment table) are recorded in
+// lf::g_device_error on the device and, through lf::g_error_mirror, in this page of
+// host memory, page-locked and mapped into the device address space.  Every entry
+// point reads it (a plain host load, no synchronization) and reports an earlier
+// call's failure before launching anything; lf_sync_status clears it.
+alignas(4096) volatile int g_host_error_page[1024];
+std::once_flag g_register_once;
+bool g_page_mapped = false;
+bool g_mirror_ready[kMaxDevices] = {};
+
+// Once per process: map the page; once per device: tell the device where it is.
+lf_status prepare_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LF_ERR_CUDA;
+    std::call_once(g_register_once, [] {
+        g_page_mapped = cudaHostRegister(const_cast<int*>(g_host_error_page), sizeof(g_host_error_page),
+                                         cudaHostRegisterMapped | cudaHostRegisterPortable) ==
+                        cudaSuccess;
+        if (!g_page_mapped) (void)cudaGetLastError();
+    });
+    std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+    if (!g_mirror_ready[dev]) {
+        int* dptr = nullptr;
+        if (g_page_mapped) {
+            void* p = nullptr;
+            if (cudaHostGetDevicePointer(&p, const_cast<int*>(g_host_error_page), 0) != cudaSuccess)
+                return LF_ERR_CUDA;
+            dptr = static_cast<int*>(p);
+        }
+        if (cudaMemcpyToSymbol(lf::g_error_mirror, &dptr, sizeof(dptr)) != cudaSuccess)
+            return LF_ERR_CUDA;
+        g_mirror_ready[dev] = true;
+    }
+    return LF_OK;
+}
+
+lf_status status_of_device_code(int code) {
+    if (code == 0) return LF_OK;
+    return (code & 0xff) == lf::kErrTimeout ? LF_ERR_TIMEOUT : LF_ERR_INVALID_ARG;
+}
+
+// An earlier call's device-side failure not yet cleared by lf_sync_status.
+lf_status pending_device_error() { return status_of_device_code(g_host_error_page[0]); }
+
 }  // namespace
 
 extern "C" {
@@ -328,7 +372,9 @@ lf_status lf_attn_fwd(const lf_attn_desc* desc, const void* q, const void* k, co
     if (!q || !k || !v || !o || !lse) return LF_ERR_INVALID_ARG;
     if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
         return LF_ERR_INVALID_ARG;
+    if ((st = pending_device_error()) != LF_OK) return st;
     if (desc->total_tokens == 0 || desc->max_seqlen == 0) return LF_OK;
+    if ((st = prepare_device()) != LF_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     return desc->d == 128 ? launch_fwd<128>(desc, q, k, v, o, lse, s)
                           : launch_fwd<64>(desc, q, k, v, o, lse, s);
@@ -356,9 +402,11 @@ static lf_status block_select_impl(const lf_attn_desc* desc, const void* dout, c
         !aligned16(tau) || !aligned16(block_weight) || !aligned16(keep) || !aligned16(kept_idx) ||
         !aligned16(kept_cnt))
         return LF_ERR_INVALID_ARG;
+    if ((st = pending_device_error()) != LF_OK) return st;
     if (desc->max_seqlen == 0) return LF_OK;
     const int nbmax = nbmax_of(desc);
     if ((size_t)nbmax * sizeof(double) > 200 * 1024) return LF_ERR_UNSUPPORTED;
+    if ((st = prepare_device()) != LF_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int write_norms = (flags & LF_SELECT_NORMS_GIVEN) ? 0 : 1;
     st = desc->d == 128 ? launch_norms<128>(desc, dout, o, block_norm, D, write_norms, s)
@@ -415,8 +463,10 @@ lf_status lf_attn_bwd(const lf_attn_desc* desc, const void* q, const void* k, co
     for (const void* p : ptrs)
         if (p && !aligned16(p)) return LF_ERR_INVALID_ARG;
     if ((o && !aligned16(o)) || (D && !aligned16(D))) return LF_ERR_INVALID_ARG;
+    if ((st = pending_device_error()) != LF_OK) return st;
     if (desc->total_tokens == 0 || desc->max_seqlen == 0) return LF_OK;
     if (!ws || ws_bytes < bwd_ws_bytes(desc, D == nullptr)) return LF_ERR_WORKSPACE;
+    if ((st = prepare_device()) != LF_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const float* Dv = D;
     if (!Dv) {
@@ -449,7 +499,9 @@ lf_status lf_attn_bwd_static_ws(const lf_attn_desc* desc, const void* q, const v
     if ((o && !aligned16(o)) || (D && !aligned16(D))) return LF_ERR_INVALID_ARG;
     const size_t need = bwd_ws_bytes(desc, D == nullptr);
     if (need > LF_STATIC_WS_BYTES) return LF_ERR_WORKSPACE;
+    if ((st = pending_device_error()) != LF_OK) return st;
     if (desc->total_tokens == 0 || desc->max_seqlen == 0) return LF_OK;
+    if ((st = prepare_device()) != LF_OK) return st;
     void* ws = nullptr;
     st = static_ws_address(&ws);
     if (st != LF_OK) return st;
@@ -471,22 +523,31 @@ lf_status lf_attn_bwd_static_ws(const lf_attn_desc* desc, const void* q, const v
 
 lf_status lf_watchdog_selftest(uint32_t limit_log2, lf_stream_t stream) {
     if (limit_log2 < 10 || limit_log2 > 31) return LF_ERR_INVALID_ARG;
+    lf_status st = pending_device_error();
+    if (st != LF_OK) return st;
+    if ((st = prepare_device()) != LF_OK) return st;
     lf::watchdog_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
         1ll << limit_log2);
     return launch_status();
 }
 
-lf_status lf_check_device_error(lf_stream_t stream) {
+lf_status lf_sync_status(lf_stream_t stream) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     if (cudaStreamSynchronize(s) != cudaSuccess) return LF_ERR_CUDA;
     int flag = 0;
     if (cudaMemcpyFromSymbol(&flag, lf::g_device_error, sizeof(int)) != cudaSuccess)
         return LF_ERR_CUDA;
-    if (flag == 0) return LF_OK;
-    const int zero = 0;
-    if (cudaMemcpyToSymbol(lf::g_device_error, &zero, sizeof(int)) != cudaSuccess)
-        return LF_ERR_CUDA;
-    return (flag & 0xff) == lf::kErrTimeout ? LF_ERR_TIMEOUT : LF_ERR_INVALID_ARG;
+    if (flag != 0) {
+        const int zero = 0;
+        if (cudaMemcpyToSymbol(lf::g_device_error, &zero, sizeof(int)) != cudaSuccess)
+            return LF_ERR_CUDA;
+    }
+    // the page may also hold a failure recorded on another device
+    const int host = g_host_error_page[0];
+    g_host_error_page[0] = 0;
+    return status_of_device_code(flag != 0 ? flag : host);
 }
+
+lf_status lf_check_device_error(lf_stream_t stream) { return lf_sync_status(stream); }
 
 }  // extern "C"

@@ -16,6 +16,9 @@ namespace lf {
 // this flag and the kernel unwinds instead of hanging the GPU.
 // ---------------------------------------------------------------------------
 __device__ int g_device_error;   // 0 = fine; otherwise (site << 8) | kind
+// Host-mapped copy of the first error (or null): lets every later host call see a
+// device-side failure without synchronizing.  Set once per device by the host.
+__device__ int* g_error_mirror;
 
 constexpr int kErrTimeout = 1;        // a bounded wait expired
 constexpr int kErrBadSegments = 2;    // cu_seqlens inconsistent with T / max_seqlen
@@ -23,7 +26,14 @@ constexpr int kErrBadSegments = 2;    // cu_seqlens inconsistent with T / max_se
 constexpr long long kWaitLimitCycles = 1ll << 31;   // ~1.1 s at 1.9 GHz
 
 __device__ __forceinline__ void report_error(int site, int kind) {
-    atomicCAS(&g_device_error, 0, (site << 8) | kind);
+    const int code = (site << 8) | kind;
+    if (atomicCAS(&g_device_error, 0, code) == 0) {
+        int* m = g_error_mirror;
+        if (m) {
+            *reinterpret_cast<volatile int*>(m) = code;
+            __threadfence_system();
+        }
+    }
 }
 __device__ __forceinline__ void report_timeout(int site) { report_error(site, kErrTimeout); }
 

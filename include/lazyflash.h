@@ -35,9 +35,22 @@
  *   Ordering: every call only enqueues work on `stream` and returns.
  *   Errors: argument errors are returned synchronously, before anything is
  *     launched (LF_ERR_INVALID_ARG, LF_ERR_UNSUPPORTED, LF_ERR_WORKSPACE).
- *     A failed launch returns LF_ERR_CUDA.  A kernel whose bounded wait expired
- *     records it in a device flag instead of hanging; lf_check_device_error
- *     synchronizes the stream and returns LF_ERR_TIMEOUT in that case.
+ *     A failed launch returns LF_ERR_CUDA.  Kernels never hang: a kernel whose
+ *     bounded wait expired (LF_ERR_TIMEOUT), or that found cu_seqlens
+ *     inconsistent with total_tokens / max_seqlen (LF_ERR_INVALID_ARG), records
+ *     the failure in a device flag and returns.  The failure is reported
+ *     (1) by the next call of any entry point made after the failing kernel
+ *     finished: the library mirrors the flag into a page of host memory mapped
+ *     into the device, so this check needs no synchronization; that call
+ *     returns the code and launches nothing; every later call does the same
+ *     until the failure is cleared; and (2) by lf_sync_status (alias
+ *     lf_check_device_error), which synchronizes the stream, returns the code
+ *     and clears it.  The flag is one per process, shared by all streams and
+ *     devices: it reports a failure of any earlier call, not only of the
+ *     caller's stream.
+ *   Set-up: the first call that launches work on a device maps the host page
+ *     (once per process) and stores its device address on that device (a
+ *     synchronous copy); make that first call before any stream capture.
  *   Thread safety: calls are reentrant; concurrent calls on different streams
  *     must use different workspaces and outputs.
  */
@@ -174,8 +187,11 @@ lf_status lf_attn_bwd(const lf_attn_desc* desc, const void* q, const void* k, co
  *   three parts rounded up to 256), plus 4 * total_tokens * hq when D is NULL,
  *   returns LF_ERR_WORKSPACE before anything is launched.
  *   The first call on a device looks up the array's device address
- *   (cudaGetSymbolAddress, with that device current); make that first call
- *   before any stream capture.  The call never calls cudaMalloc, cudaFree or an
+ *   (cudaGetSymbolAddress, with that device current) and keeps it for the life
+ *   of the process; make that first call before any stream capture.  A device
+ *   reset (cudaDeviceReset, or a framework that destroys and recreates the
+ *   primary context) reloads the library's device code, possibly at another
+ *   address: do not call this entry point on a device after resetting it.  The call never calls cudaMalloc, cudaFree or an
  *   allocating library routine; the accumulators a call uses are cleared at
  *   its start (dK and dV need none when the query heads of each KV head fit
  *   in one CTA, i.e. hq/hkv is 1, 2 or 4: they are then written directly).
@@ -196,9 +212,17 @@ lf_status lf_attn_bwd_static_ws(const lf_attn_desc* desc, const void* q, const v
  * Returns LF_ERR_INVALID_ARG for a limit outside 10..31. */
 lf_status lf_watchdog_selftest(uint32_t limit_log2, lf_stream_t stream);
 
-/* Waits for `stream`, then reads and clears the device watchdog flag.
- * LF_ERR_TIMEOUT if a kernel gave up a bounded wait since the last check,
- * LF_ERR_CUDA if the stream reported an error, else LF_OK. */
+/* Waits for `stream`, then reads and clears the device-side failure flag (see
+ * "Errors" above).  Returns LF_ERR_TIMEOUT if a kernel gave up a bounded wait
+ * since the flag was last cleared, LF_ERR_INVALID_ARG if a kernel found
+ * cu_seqlens inconsistent with total_tokens / max_seqlen (the first failure is
+ * the one reported), LF_ERR_CUDA if the stream reported a CUDA error, else
+ * LF_OK.  The flag is shared by all streams and devices of the process, so a
+ * check on one stream also reports, and clears, a failure raised by a kernel on
+ * another stream. */
+lf_status lf_sync_status(lf_stream_t stream);
+
+/* The same function as lf_sync_status (its earlier name). */
 lf_status lf_check_device_error(lf_stream_t stream);
 
 /* Static, human-readable name of a status code. */

@@ -1,4 +1,4 @@
-"""Failure detection without a GPU fault (survey section 5): every wait in the
+"""Failure detection without a GPU fault: every wait in the
 kernels is bounded; when one runs out the kernel records it in a device flag
 and returns, and the host reads LF_ERR_TIMEOUT.  The self-test makes a wait run
 out (a barrier phase that nothing completes) and checks that the status comes
@@ -33,3 +33,33 @@ def test_expired_wait_is_reported_and_context_survives():
     w = synthetic.TINY
     _, _, bufs = run_step(w)
     assert torch.isfinite(bufs.dq.float()).all() and torch.isfinite(bufs.o.float()).all()
+
+
+@pytest.mark.gpu
+def test_next_call_reports_the_expired_wait_without_a_sync():
+    """An expired wait is reported by the next call of any entry point (which then
+    launches nothing) until lf_sync_status clears it."""
+    lf.lf_sync_status()
+    w = synthetic.TINY
+    inp = synthetic.make_inputs(w)
+    desc, dev, bufs = run_step(w, inp)
+    lf.lf_watchdog_selftest(22)
+    torch.cuda.synchronize()                    # the failing kernel has finished
+    marker = torch.full_like(bufs.o, 7.0)
+    for _ in range(2):                          # every call until cleared
+        with pytest.raises(lf.LfError) as ei:
+            lf.lf_attn_fwd(desc, dev["q"], dev["k"], dev["v"], marker, bufs.lse)
+        assert ei.value.code == lf.LF_ERR_TIMEOUT
+    torch.cuda.synchronize()
+    assert torch.all(marker == 7.0)             # nothing was launched
+    with pytest.raises(lf.LfError) as ei:
+        lf.lf_attn_bwd(desc, dev["q"], dev["k"], dev["v"], bufs.o, bufs.lse, dev["dout"], bufs.D,
+                       bufs.w, bufs.kept_idx, bufs.kept_cnt, bufs.dq, bufs.dk, bufs.dv, bufs.ws)
+    assert ei.value.code == lf.LF_ERR_TIMEOUT
+    with pytest.raises(lf.LfError) as ei:
+        lf.lf_sync_status()
+    assert ei.value.code == lf.LF_ERR_TIMEOUT
+    lf.lf_sync_status()                         # cleared
+    lf.lf_attn_fwd(desc, dev["q"], dev["k"], dev["v"], marker, bufs.lse)
+    lf.lf_sync_status()
+    assert torch.equal(marker, bufs.o)

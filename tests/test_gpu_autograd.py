@@ -8,15 +8,17 @@ import torch
 import torch.nn.functional as F
 
 import block_sparse_attention_dense_b200 as lf
+import oracle
 from block_sparse_attention_dense_b200.autograd import lazyflash_attention
 import synthetic
-from _helpers import rel_fro, run_step
+from _helpers import nb_per_seq, rel_fro, run_step
 
 pytestmark = pytest.mark.gpu
 
 
 def _reference(q, k, v, cu, dout):
-    """fp32 torch attention per segment (the reference the survey names)."""
+    """fp32 torch attention per segment: the plain PyTorch reference of the dense
+    attention gradient."""
     q = q.float().detach().requires_grad_(True)
     k = k.float().detach().requires_grad_(True)
     v = v.float().detach().requires_grad_(True)
@@ -63,3 +65,38 @@ def test_autograd_steps_draw_fresh_masks():
         o.backward(dev["dout"])
         grads.append(q.grad.clone())
     assert not torch.equal(grads[0], grads[1])
+
+
+def test_autograd_at_positive_delta_matches_the_oracle():
+    """delta > 0 through the autograd wrapper: the selection it drew equals the
+    oracle's on the GPU's block norms (bit-exact), and the gradients equal the
+    oracle's reweighted gradient for that draw (article section "Un budget sur la
+    masse de gradient, et un tirage qui garde le gradient non biaisé": the estimate
+    is the dense gradient of the kept blocks' output gradients times 1/p)."""
+    w = synthetic.Workload("ag_delta", (700, 300), hq=4, hkv=2, d=128, block=128, sigma=2.0,
+                           delta=0.2)
+    inp = synthetic.make_inputs(w)
+    dev = {k_: t.cuda() for k_, t in inp.items()}
+    q = dev["q"].clone().requires_grad_(True)
+    k = dev["k"].clone().requires_grad_(True)
+    v = dev["v"].clone().requires_grad_(True)
+    sel_gpu = {}
+    o = lazyflash_attention(q, k, v, dev["cu_seqlens"], w.max_seqlen, delta=w.delta, seed=9,
+                            step=4, selection_out=sel_gpu)
+    o.backward(dev["dout"])
+    lf.lf_check_device_error()
+    assert sel_gpu["step"] == 4
+    nb = nb_per_seq(w)
+    sel = oracle.select(sel_gpu["norm"].cpu().numpy(), nb, w.delta, 9, 4)
+    np.testing.assert_array_equal(sel_gpu["keep"].cpu().numpy(), sel["keep"])
+    np.testing.assert_array_equal(sel_gpu["weight"].cpu().numpy().view(np.uint32),
+                                  sel["w"].view(np.uint32))
+    np.testing.assert_array_equal(sel_gpu["tau"].cpu().numpy().view(np.uint64),
+                                  sel["tau"].view(np.uint64))
+    kept = sel["keep"][:, :, : int(nb.max())]
+    assert 0 < kept.sum() < kept.size        # a real sparse draw
+    dq_ref, dk_ref, dv_ref = oracle.attn_bwd(w.cu_seqlens(), inp["q"], inp["k"], inp["v"],
+                                             inp["dout"], w.scale, w.block,
+                                             sel["w"].astype(np.float64), True)
+    for got, ref in ((q.grad, dq_ref), (k.grad, dk_ref), (v.grad, dv_ref)):
+        assert rel_fro(got.float().cpu().numpy(), ref) < 1e-2

@@ -40,6 +40,10 @@ SMALL = [
     # accumulators; the forward's head-in-group index with an odd group
     synthetic.Workload("gqa3_d128", (333, 200), hq=6, hkv=2, d=128, block=128, sigma=1.5,
                        delta=0.1),
+    # 60 segments: the forward's segment search takes its multi-round path (more than 32
+    # segment starts) and meets empty, one-token and tile-edge lengths (127, 128, 129, 256)
+    synthetic.Workload("many_segments", (0, 1, 127, 128, 129, 256, 300, 5, 64, 200) * 6, hq=2,
+                       hkv=1, d=64, block=64, sigma=1.5, delta=0.2),
 ]
 
 
@@ -275,8 +279,32 @@ LONG_D64 = synthetic.Workload("long_d64", (262144,), hq=2, hkv=1, d=64, block=64
                               delta=0.1)
 
 
-@pytest.mark.parametrize("w", [synthetic.HEADLINE, synthetic.VARLEN, LONG_D64], ids=lambda w: w.name)
-def test_full_size_sampled_parity(w):
+def _kv_tile_rows(w, cu, kv_tile):
+    """Sampled KV rows of one KV tile for the dK/dV check: "first" is KV tile 0 of
+    the longest segment, whose walk is the longest of the launch (under the causal
+    mask every kept query tile of the segment reaches it: many work-list ring and
+    pipeline-phase wraps, and the longest accumulation in tensor memory); "last" is
+    the segment-final tile of the last segment (the shortest walk).  Returns (rows,
+    kv heads)."""
+    lens = np.diff(cu)
+    if kv_tile == "first":
+        s = int(np.argmax(lens))
+        u0, u1 = int(cu[s]), int(cu[s]) + 128
+        rows = np.arange(u0, u1, 8, dtype=np.int32)
+        heads = np.zeros(len(rows), dtype=np.int32)     # one KV head: one LSE pass
+    else:
+        s = w.nseq - 1
+        u0 = max(int(cu[s + 1]) - 128, int(cu[s]))
+        rows = np.arange(u0, int(cu[s + 1]), 8, dtype=np.int32)
+        heads = (np.arange(len(rows)) % w.hkv).astype(np.int32)
+    return rows, heads
+
+
+@pytest.mark.parametrize("w,kv_tile", [
+    (synthetic.HEADLINE, "first"), (synthetic.LONG, "first"), (synthetic.VARLEN, "first"),
+    (LONG_D64, "last"),
+], ids=["headline", "long", "varlen", "long_d64"])
+def test_full_size_sampled_parity(w, kv_tile):
     inp = synthetic.make_inputs(w)
     desc, dev, bufs = run_step(w, inp)
     cu = w.cu_seqlens()
@@ -307,8 +335,8 @@ def test_full_size_sampled_parity(w):
     lse = _cpu(bufs.lse)[heads, rows]
     assert np.abs(o - o_ref).max() < O_TOL
     assert np.abs(lse - lse_ref).max() < LSE_TOL
-    # backward: dQ at sampled rows of kept blocks, zero at dropped blocks;
-    # dK/dV at the last KV tile of one segment (cheap for the row oracle)
+    # backward: dQ at sampled rows of kept blocks, zero at dropped blocks; dK/dV at
+    # sampled rows of one KV tile (see _kv_tile_rows)
     wb = sel["w"].astype(np.float64)
     kept_rows, kept_heads = [], []
     dq = bufs.dq.cpu()
@@ -323,10 +351,17 @@ def test_full_size_sampled_parity(w):
                 kept_heads.append(h)
         else:
             assert torch.all(dq[t, h] == 0)
-    s_last = w.nseq - 1
-    u0 = max(int(cu[s_last + 1]) - 128, int(cu[s_last]))
-    kv_rows = np.arange(u0, int(cu[s_last + 1]), 8, dtype=np.int32)
-    kv_heads = (np.arange(len(kv_rows)) % w.hkv).astype(np.int32)
+    kv_rows, kv_heads = _kv_tile_rows(w, cu, kv_tile)
+    if kv_tile == "first":
+        # the walk checked is long: count the kept (head, query tile) pairs it visits
+        s0 = int(np.searchsorted(cu, kv_rows[0], side="right") - 1)
+        G = w.hq // w.hkv
+        per = 128 // w.block
+        kept_tiles = sel["keep"][s0, :G, : nb[s0]]
+        ntile = (nb[s0] + per - 1) // per
+        walked = sum(int(kept_tiles[h, i * per:(i + 1) * per].any()) for h in range(G)
+                     for i in range(ntile))
+        assert walked >= 40, walked
     dq_ref, dk_ref, dv_ref = oracle.attn_bwd_rows(cu, inp["q"], inp["k"], inp["v"], dout, w.scale,
                                                   w.block, wb, kept_rows, kept_heads, kv_rows,
                                                   kv_heads)
@@ -338,6 +373,60 @@ def test_full_size_sampled_parity(w):
         assert rel_fro(dv, dv_ref) < GRAD_TOL
     else:
         assert np.all(dk == 0) and np.all(dv == 0)
+
+
+def test_gqa_mid_full_oracle():
+    """The GQA-mid workload (4096 tokens, 32 query heads over 8 KV heads, d = 128,
+    delta = 0.05) against the full oracle: every output element."""
+    w = synthetic.GQA_MID
+    inp = synthetic.make_inputs(w)
+    desc, dev, bufs = run_step(w, inp, seed=4, step=7)
+    cu = w.cu_seqlens()
+    nb = nb_per_seq(w)
+    o_ref, lse_ref = oracle.attn_fwd(cu, inp["q"], inp["k"], inp["v"], w.scale, w.causal)
+    assert np.abs(_cpu(bufs.o) - o_ref).max() < O_TOL
+    assert np.abs(_cpu(bufs.lse) - lse_ref).max() < LSE_TOL
+    m_ref = oracle.block_norms(cu, inp["dout"], w.block, w.nbmax)
+    m = _cpu(bufs.norm)
+    assert np.all(np.abs(m - m_ref) <= NORM_TOL * np.maximum(m_ref, 1e-30))
+    D_ref = oracle.rowdot(inp["dout"], bufs.o.cpu())
+    scale = np.sqrt(oracle.rowdot(inp["dout"], inp["dout"]) * oracle.rowdot(bufs.o.cpu(), bufs.o.cpu()))
+    assert np.all(np.abs(_cpu(bufs.D) - D_ref) <= 1e-5 * scale + 1e-30)
+    sel = oracle.select(m, nb, w.delta, 4, 7)
+    np.testing.assert_array_equal(bufs.tau.cpu().numpy().view(np.uint64), sel["tau"].view(np.uint64))
+    np.testing.assert_array_equal(bufs.keep.cpu().numpy(), sel["keep"])
+    np.testing.assert_array_equal(bufs.w.cpu().numpy().view(np.uint32), sel["w"].view(np.uint32))
+    np.testing.assert_array_equal(bufs.kept_idx.cpu().numpy(), sel["kept_idx"])
+    np.testing.assert_array_equal(bufs.kept_cnt.cpu().numpy(), sel["kept_cnt"])
+    assert 0 < sel["keep"].mean() < 1
+    dq_ref, dk_ref, dv_ref = oracle.attn_bwd(cu, inp["q"], inp["k"], inp["v"], inp["dout"], w.scale,
+                                             w.block, sel["w"].astype(np.float64), w.causal)
+    assert rel_fro(_cpu(bufs.dq), dq_ref) < GRAD_TOL
+    assert rel_fro(_cpu(bufs.dk), dk_ref) < GRAD_TOL
+    assert rel_fro(_cpu(bufs.dv), dv_ref) < GRAD_TOL
+
+
+@pytest.mark.parametrize("w", [SMALL[1], SMALL[4]], ids=lambda w: w.name)
+def test_backward_computes_D_itself(w):
+    """lf_attn_bwd with D = NULL computes D = rowsum(dO * O) from o and dout in its
+    workspace; the gradients match those computed with the selection's D."""
+    inp = synthetic.make_inputs(w)
+    desc, dev, bufs = run_step(w, inp, seed=3, step=1)
+    ref = {k: getattr(bufs, k).float().cpu() for k in ("dq", "dk", "dv")}
+    out = {k: torch.full_like(getattr(bufs, k), float("nan")) for k in ("dq", "dk", "dv")}
+    lf.lf_attn_bwd(desc, dev["q"], dev["k"], dev["v"], bufs.o, bufs.lse, dev["dout"], None, bufs.w,
+                   bufs.kept_idx, bufs.kept_cnt, out["dq"], out["dk"], out["dv"], bufs.ws)
+    lf.lf_check_device_error()
+    sel = oracle.select(_cpu(bufs.norm), nb_per_seq(w), w.delta, 3, 1)
+    dq_ref, dk_ref, dv_ref = oracle.attn_bwd(w.cu_seqlens(), inp["q"], inp["k"], inp["v"],
+                                             inp["dout"], w.scale, w.block,
+                                             sel["w"].astype(np.float64), w.causal)
+    for k, oref in (("dq", dq_ref), ("dk", dk_ref), ("dv", dv_ref)):
+        got = out[k].float().cpu()
+        assert torch.isfinite(got).all(), k
+        assert rel_fro(got, oref) < GRAD_TOL, k
+        # the same gradients as with the selection's D, up to the rounding of the sums
+        assert rel_fro(got, ref[k]) < 1e-3, k
 
 
 @pytest.mark.parametrize("case", [

@@ -19,11 +19,12 @@ from _helpers import rel_fro, run_step
 GRAD_TOL = 1e-2   # the backward parity tolerance of the other GPU tests
 
 
-# two query heads per KV head: dK/dV written directly by whole-group CTAs; three: dK/dV
-# through the fp32 accumulators in the static array
+# two and three query heads per KV head (two group sizes of the backward's CTAs), each with
+# the selection's D and with D computed by the call itself
 @pytest.mark.gpu
-@pytest.mark.parametrize("hq", [4, 6], ids=["group2_direct", "group3_accumulators"])
-def test_static_scratch_backward_matches_workspace_backward_twice(hq):
+@pytest.mark.parametrize("D_given", [True, False], ids=["D_given", "D_computed"])
+@pytest.mark.parametrize("hq", [4, 6], ids=["group2", "group3"])
+def test_static_scratch_backward_matches_workspace_backward_twice(hq, D_given):
     w = synthetic.Workload("no_alloc", (700, 300), hq=hq, hkv=2, d=128, block=128, sigma=1.5,
                            delta=0.1)
     # one full step through the ordinary entry points (caller workspace)
@@ -33,9 +34,10 @@ def test_static_scratch_backward_matches_workspace_backward_twice(hq):
     assert need <= 32 << 20
     for call in range(2):
         out = {k: torch.full_like(getattr(bufs, k), float("nan")) for k in ("dq", "dk", "dv")}
+        # without D, the call computes it from o and dout in the static array too
         lf.lf_attn_bwd_static_ws(desc, dev["q"], dev["k"], dev["v"], bufs.o, bufs.lse,
-                                 dev["dout"], bufs.D, bufs.w, bufs.kept_idx, bufs.kept_cnt,
-                                 out["dq"], out["dk"], out["dv"])
+                                 dev["dout"], bufs.D if D_given else None, bufs.w, bufs.kept_idx,
+                                 bufs.kept_cnt, out["dq"], out["dk"], out["dv"])
         lf.lf_check_device_error()
         torch.cuda.synchronize()
         for k in ("dq", "dk", "dv"):
