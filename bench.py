@@ -71,6 +71,47 @@ def tile_flops(w: synthetic.Workload, keep=None):
     return fwd, bwd_dense, bwd_exec
 
 
+def selection_telemetry(w: synthetic.Workload, norm, tau, keep, bwd_exec_fl, bwd_dense_fl):
+    """What the selection did, per (segment, head), from the GPU's outputs: the
+    kept fraction of blocks, tau, and the expected discarded share
+    sum_b (1 - p_b) m_b / sum_b m_b with p_b = min(1, m_b / tau), which the budget
+    bounds by delta (article sections "Un budget sur la masse de gradient ..." and
+    "Le choix des blocs pèse plus que la quantité sautée")."""
+    kept_frac, taus, shares = [], [], []
+    n_kept = n_all = 0
+    for s, L in enumerate(w.seqlens):
+        nb = (L + w.block - 1) // w.block
+        if nb == 0:
+            continue
+        for h in range(w.hq):
+            m = norm[s, h, :nb].astype(np.float64)
+            k = keep[s, h, :nb]
+            n_kept += int(k.sum())
+            n_all += nb
+            kept_frac.append(float(k.mean()))
+            t = float(tau[s, h])
+            taus.append(t)
+            tot = m.sum()
+            if t > 0 and tot > 0:
+                p = np.minimum(1.0, m / t)
+                shares.append(float(((1.0 - p) * m).sum() / tot))
+            else:
+                shares.append(0.0)
+
+    def mmm(x):
+        return {"min": float(np.min(x)), "median": float(np.median(x)), "max": float(np.max(x))}
+
+    return {"kept_fraction": n_kept / max(1, n_all),
+            "kept_fraction_per_head": mmm(kept_frac),
+            "tau": mmm(taus),
+            "expected_discarded_share": {"max": float(np.max(shares)),
+                                         "median": float(np.median(shares)),
+                                         "bound_delta": w.delta,
+                                         "within_bound": bool(np.max(shares) <= w.delta + 1e-12)},
+            "executed_vs_dense_flops": bwd_exec_fl / bwd_dense_fl,
+            "heads": len(kept_frac)}
+
+
 # ---------------------------------------------------------------------------
 # clocks during the timed region
 # ---------------------------------------------------------------------------
@@ -207,7 +248,8 @@ def kernels_per_step(w: synthetic.Workload) -> int:
 def oracle_sample(w: synthetic.Workload, inp, prefix: int, seed=0, step=0):
     """The oracle's forward, selection and weighted backward on the first
     `prefix` tokens of segment 0 (a causal prefix is itself a complete problem),
-    all heads.  Returns (seconds, executed tile FLOPs of the sample, threads)."""
+    all heads.  Returns a dict: seconds of the backward and of the whole step,
+    the sample's executed backward tile FLOPs and step FLOPs, and the threads."""
     import oracle
     ws = w.with_(seqlens=(prefix,))
     sl = slice(0, prefix)
@@ -218,11 +260,13 @@ def oracle_sample(w: synthetic.Workload, inp, prefix: int, seed=0, step=0):
     o, lse = oracle.attn_fwd(cu, q, k, v, ws.scale, ws.causal)
     m = oracle.block_norms(cu, do, ws.block)
     sel = oracle.select(m, oracle.nblocks(cu, ws.block), ws.delta, seed, step)
+    t1 = time.perf_counter()
     oracle.attn_bwd(cu, q, k, v, do, ws.scale, ws.block, sel["w"].astype(np.float64), ws.causal)
-    dt = time.perf_counter() - t0
+    t2 = time.perf_counter()
     f, _, b = tile_flops(ws, sel["keep"])
     threads = int(os.environ.get("OMP_NUM_THREADS", len(os.sched_getaffinity(0))))
-    return dt, f + b, threads
+    return {"bwd_s": t2 - t1, "step_s": t2 - t0, "bwd_flops": b, "step_flops": f + b,
+            "threads": threads}
 
 
 def max_over_ranks(values, dist=None, device=None):
@@ -248,19 +292,22 @@ def run_reference(args, w, rank):
     inp = synthetic.make_inputs(w, rows=prefix) if w.nseq == 1 else synthetic.make_inputs(w)
     for _ in range(args.warmup):
         oracle_sample(w, inp, prefix)
-    tot_t = tot_f = 0.0
+    tot_b = tot_s = tot_f = 0.0
     threads = 1
     for _ in range(args.steps):
-        dt, fl, threads = oracle_sample(w, inp, prefix)
-        tot_t += dt
-        tot_f += fl
-    val = tot_f / tot_t / 1e12
-    sample = ("oracle fwd+select+bwd on the first %d tokens of the %s workload, all %d heads "
-              "(a causal prefix is a complete sub-problem)" % (prefix, w.name, w.hq))
+        r = oracle_sample(w, inp, prefix)
+        tot_b += r["bwd_s"]
+        tot_s += r["step_s"]
+        tot_f += r["bwd_flops"]
+        threads = r["threads"]
+    val = tot_f / tot_b / 1e12
+    sample = ("oracle backward (its executed tile FLOPs over its own time; the forward and "
+              "selection that feed it run untimed) on the first %d tokens of the %s workload, "
+              "all %d heads (a causal prefix is a complete sub-problem)" % (prefix, w.name, w.hq))
     line = {
         "impl": "reference", "metric": args.metric, "value": val, "unit": "TFLOP/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
-        "ms_per_step": 1e3 * tot_t / args.steps, "higher_is_better": True, "scaling": "weak",
+        "ms_per_step": 1e3 * tot_s / args.steps, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": config_of(w, args),
         "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
@@ -384,6 +431,8 @@ def main():
     ap.add_argument("--ref-prefix", type=int, default=1024,
                     help="tokens of the oracle sample timed per step by --impl reference")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-dense-arm", action="store_true",
+                    help="skip the delta = 0 comparison run after the timed region")
     ap.add_argument("--layers", type=int, default=0,
                     help="time the synthetic layer-stack step instead (its own JSON line)")
     args = ap.parse_args()
@@ -433,55 +482,79 @@ def main():
                         w.block)
     bufs = lf.Buffers(desc, device=dev)
 
-    def select():
-        lf.lf_block_select_rule(desc, d_in["dout"], bufs.o, rule_id, rule_param, 0, 0, 0, bufs.norm,
+    def select(param):
+        lf.lf_block_select_rule(desc, d_in["dout"], bufs.o, rule_id, param, 0, 0, 0, bufs.norm,
                                 bufs.D, bufs.tau, bufs.w, bufs.keep, bufs.kept_idx, bufs.kept_cnt)
 
-    def step():
+    def step(param):
         lf.lf_attn_fwd(desc, d_in["q"], d_in["k"], d_in["v"], bufs.o, bufs.lse)
-        select()
+        select(param)
         lf.lf_attn_bwd(desc, d_in["q"], d_in["k"], d_in["v"], bufs.o, bufs.lse, d_in["dout"],
                        bufs.D, bufs.w, bufs.kept_idx, bufs.kept_cnt, bufs.dq, bufs.dk, bufs.dv,
                        bufs.ws)
 
+    def timed_region(K, param):
+        """K steps back to back on `stream`, CUDA events around the region and around
+        each phase; returns (region ms, summed fwd, select and bwd ms)."""
+        ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for i in range(K):
+            e = ev[i]
+            e[0].record(stream)
+            lf.lf_attn_fwd(desc, d_in["q"], d_in["k"], d_in["v"], bufs.o, bufs.lse)
+            e[1].record(stream)
+            select(param)
+            e[2].record(stream)
+            lf.lf_attn_bwd(desc, d_in["q"], d_in["k"], d_in["v"], bufs.o, bufs.lse, d_in["dout"],
+                           bufs.D, bufs.w, bufs.kept_idx, bufs.kept_cnt, bufs.dq, bufs.dk, bufs.dv,
+                           bufs.ws)
+            e[3].record(stream)
+        end.record(stream)
+        torch.cuda.synchronize()
+        return (start.elapsed_time(end), sum(e[0].elapsed_time(e[1]) for e in ev),
+                sum(e[1].elapsed_time(e[2]) for e in ev), sum(e[2].elapsed_time(e[3]) for e in ev))
+
     for _ in range(max(3, args.warmup)):
-        step()
-    lf.lf_check_device_error()
+        step(rule_param)
+    lf.lf_sync_status()
     torch.cuda.synchronize()
     keep = bufs.keep.cpu().numpy()
     fwd_fl, bwd_dense_fl, bwd_exec_fl = tile_flops(w, keep)
+    telemetry = selection_telemetry(w, bufs.norm.cpu().numpy(), bufs.tau.cpu().numpy(), keep,
+                                    bwd_exec_fl, bwd_dense_fl)
 
     # ---- device-timed steps, inputs resident; per-phase events on the launching stream
     K = args.steps
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
     if dist is not None:
         dist.barrier()
     torch.cuda.synchronize()
     clocks = ClockSampler(local)
-    start = torch.cuda.Event(enable_timing=True)
-    end = torch.cuda.Event(enable_timing=True)
-    start.record(stream)
-    for i in range(K):
-        e = ev[i]
-        e[0].record(stream)
-        lf.lf_attn_fwd(desc, d_in["q"], d_in["k"], d_in["v"], bufs.o, bufs.lse)
-        e[1].record(stream)
-        select()
-        e[2].record(stream)
-        lf.lf_attn_bwd(desc, d_in["q"], d_in["k"], d_in["v"], bufs.o, bufs.lse, d_in["dout"],
-                       bufs.D, bufs.w, bufs.kept_idx, bufs.kept_cnt, bufs.dq, bufs.dk, bufs.dv,
-                       bufs.ws)
-        e[3].record(stream)
-    end.record(stream)
-    torch.cuda.synchronize()
+    total_ms, fwd_sum, sel_sum, bwd_sum = timed_region(K, rule_param)
     if dist is not None:
         dist.barrier()
     clk = clocks.stop()
-    total_ms = start.elapsed_time(end)
-    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in ev) / K
-    sel_ms = sum(e[1].elapsed_time(e[2]) for e in ev) / K
-    bwd_ms = sum(e[2].elapsed_time(e[3]) for e in ev) / K
-    lf.lf_check_device_error()
+    fwd_ms, sel_ms, bwd_ms = fwd_sum / K, sel_sum / K, bwd_sum / K
+    lf.lf_sync_status()
+
+    # ---- the dense backward (delta = 0) through the same kernels: does the backward's
+    # time follow the executed fraction?  (article section "A 32 000 tokens, 5,72 fois")
+    dense_arm = None
+    if rule_id == 0 and w.delta > 0 and not args.no_dense_arm:
+        K0 = max(3, K // 2)
+        for _ in range(2):
+            step(0.0)
+        torch.cuda.synchronize()
+        if dist is not None:
+            dist.barrier()
+        _, _, _, bwd0_sum = timed_region(K0, 0.0)
+        lf.lf_sync_status()
+        bwd0_ms = max_over_ranks([bwd0_sum / K0], dist, dev)[0]
+        dense_arm = {"delta": 0.0, "steps": K0, "bwd_ms": bwd0_ms,
+                     "bwd_tflops": bwd_dense_fl / (bwd0_ms * 1e-3) / 1e12}
+        step(rule_param)          # leave the workload's own selection in the buffers
+        torch.cuda.synchronize()
 
     # ---- end to end through the API: host inputs in, results out, every step.  The
     # copies run on two side streams with double-buffered device inputs and outputs,
@@ -546,18 +619,24 @@ def main():
     e2e_ms = e2s.elapsed_time(e2e)
     lf.lf_check_device_error()
 
-    # ---- max over ranks
-    total_ms, e2e_ms = max_over_ranks([total_ms, e2e_ms], dist, dev)
+    # ---- max over ranks (the job is as slow as its slowest rank)
+    total_ms, bwd_sum, e2e_ms = max_over_ranks([total_ms, bwd_sum, e2e_ms], dist, dev)
+    bwd_ms = bwd_sum / K
 
     n = world
     step_fl = fwd_fl + bwd_exec_fl
-    value = whole_job_tflops(n, K, step_fl, total_ms)
-    e2e_val = whole_job_tflops(n, Ke, step_fl, e2e_ms)
+    # the metric: the LazyFlash backward's executed FLOPs per second, whole job
+    value = whole_job_tflops(n, K, bwd_exec_fl, bwd_sum)
+    # end to end: the same backward FLOPs per second of data-fed step time (fwd, select,
+    # bwd, host copies in and out)
+    e2e_val = whole_job_tflops(n, Ke, bwd_exec_fl, e2e_ms)
     peaks = _load_json(os.path.join(ROOT, "MEASURED_PEAKS.json"))
     if peaks:
-        peak, peak_src = float(peaks["bf16_tflops_sustained"]), "measured (sustained)"
+        peak, peak_burst, peak_src = (float(peaks["bf16_tflops_sustained"]),
+                                      float(peaks["bf16_tflops"]), "measured")
     else:
-        peak, peak_src = 1400.0, "fallback (sustained)"
+        peak, peak_burst, peak_src = 1400.0, 1590.0, "fallback"
+    hbm_peak = float(peaks["hbm_gbs"]) if peaks else 6650.0
     fwd_tf = fwd_fl / (fwd_ms * 1e-3) / 1e12
     bwd_tf = bwd_exec_fl / (bwd_ms * 1e-3) / 1e12
     traffic = _load_json(os.path.join(ROOT, "profiles", "traffic.json")) or {}
@@ -571,15 +650,21 @@ def main():
                 if hashlib.sha1(f.read()).hexdigest()[:12] == rec.get("source_sha1"):
                     t = rec.get("bytes_per_launch")
         return {"bound": "tensor", "kernel": kernel, "timed": call, "achieved": achieved,
-                "peak": peak, "peak_source": peak_src, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": t}
+                "peak": peak, "peak_source": peak_src + " bf16, sustained (the kernel runs inside "
+                "a long back-to-back step under the power cap)", "unit": "TFLOP/s",
+                "frac": achieved / peak, "peak_burst": peak_burst, "frac_burst": achieved / peak_burst,
+                "traffic": t}
 
     roof_fwd = roof("attn_fwd_kernel", "lf_attn_fwd (one kernel)", fwd_tf)
-    roof_bwd = roof("attn_bwd_kernel", "lf_attn_bwd (dK/dV memset, kept-rows dQ zeroing, "
-                    "attn_bwd_kernel, 3 fp32->bf16 conversions; the kernel is ~97% of the call in "
-                    "the ncu launch list)", bwd_tf)
+    roof_bwd = roof("attn_bwd_kernel", "the lf_attn_bwd call (memsets and the small dQ kernels "
+                    "around attn_bwd_kernel included; the kernel is ~97%% of the call in the ncu "
+                    "launch list); FLOPs: executed tile FLOPs of the kept query tiles", bwd_tf)
+    sel_bytes = 2 * w.total_tokens * w.hq * w.d * 2 + w.total_tokens * w.hq * 4
     line = {
-        "metric": args.metric, "value": value, "unit": "TFLOP/s", "n_gpus": n, "steps": K,
+        "metric": args.metric, "value": value, "unit": "TFLOP/s",
+        "value_is": "LazyFlash backward (lf_attn_bwd) executed TFLOP/s, whole job; "
+                    "ms_per_step is the whole step (fwd + select + bwd)",
+        "n_gpus": n, "steps": K,
         "warmup": max(3, args.warmup), "ms_per_step": total_ms / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
         "config": config_of(w, args),
@@ -587,27 +672,39 @@ def main():
         "bwd_ms": bwd_ms, "bwd_tflops_executed": bwd_tf,
         "bwd_tflops_dense_equiv": bwd_dense_fl / (bwd_ms * 1e-3) / 1e12,
         "fwd_tflops": fwd_tf,
+        "step_tflops_executed": whole_job_tflops(n, K, step_fl, total_ms),
+        "select_gbs": {"achieved": sel_bytes / (sel_ms * 1e-3) / 1e9, "peak": hbm_peak,
+                       "frac": sel_bytes / (sel_ms * 1e-3) / 1e9 / hbm_peak,
+                       "bytes": sel_bytes, "timed": "the lf_block_select call (norm pass and "
+                       "selection kernels)"},
         "flops_per_step": {"fwd": fwd_fl, "bwd_executed": bwd_exec_fl, "bwd_dense": bwd_dense_fl},
-        "kept_fraction": float(keep.astype(bool).sum() / max(1, int(sum(
-            (L + w.block - 1) // w.block for L in w.seqlens)) * w.hq)),
+        "kept_fraction": telemetry["kept_fraction"],
         "bwd_executed_fraction": bwd_exec_fl / bwd_dense_fl,
-        "roofline": roof_fwd if fwd_ms >= bwd_ms else roof_bwd,
+        "telemetry": telemetry,
+        "roofline": roof_bwd,
         "roofline_fwd": roof_fwd,
-        "roofline_bwd": roof_bwd,
         "e2e": {"value": e2e_val, "unit": "TFLOP/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / Ke, "steps": Ke,
+                "is": "backward executed FLOPs per second of data-fed step time (fwd, select, "
+                      "bwd and the host copies of inputs and results)",
                 "copies": "pinned host buffers; uploads and downloads on two side streams, "
                           "device inputs and outputs double-buffered"},
         "gpu_launches": kernels_per_step(w) * K,
         "clocks": clk,
     }
+    if dense_arm is not None:
+        dense_arm["time_ratio"] = bwd_ms / dense_arm["bwd_ms"]
+        dense_arm["executed_fraction"] = bwd_exec_fl / bwd_dense_fl
+        dense_arm["speedup"] = dense_arm["bwd_ms"] / bwd_ms
+        line["vs_delta0"] = dense_arm
     if rank == 0 and n == 1 and not args.no_cpu_baseline:
-        dt, fl, threads = oracle_sample(w, inp, min(args.cpu_prefix, w.seqlens[0]))
+        r = oracle_sample(w, inp, min(args.cpu_prefix, w.seqlens[0]))
         line["cpu_baseline"] = {
-            "value": fl / dt / 1e12, "unit": "TFLOP/s", "cores": threads, "kind": "oracle",
-            "seconds": dt,
-            "sample": "oracle fwd+select+bwd on the first %d tokens of the %s workload, all %d "
-                      "heads" % (min(args.cpu_prefix, w.seqlens[0]), w.name, w.hq)}
+            "value": r["bwd_flops"] / r["bwd_s"] / 1e12, "unit": "TFLOP/s", "cores": r["threads"],
+            "kind": "oracle", "seconds": r["step_s"], "bwd_seconds": r["bwd_s"],
+            "sample": "oracle backward (executed tile FLOPs over its time) on the first %d tokens "
+                      "of the %s workload, all %d heads; its forward and selection ran untimed"
+                      % (min(args.cpu_prefix, w.seqlens[0]), w.name, w.hq)}
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:

@@ -156,18 +156,20 @@ template <int D>
 lf_status launch_norms(const lf_attn_desc* d, const void* dout, const void* o, float* norms,
                        float* Dv, int write_norms, cudaStream_t st) {
     dim3 grid(nbmax_of(d), d->hq, d->nseq);
-    lf::norms_rowdot_kernel<D><<<grid, 128, 0, st>>>(
+    lf::norms_rowdot_kernel<D><<<grid, lf::kNormThreads, 0, st>>>(
         d->cu_seqlens, d->total_tokens, d->max_seqlen, d->hq, d->block_q, nbmax_of(d),
         static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(o), norms, Dv,
         write_norms);
     return launch_status();
 }
 
+// The backward: prologue over kept blocks (dQ accumulator rows zeroed; D computed into
+// the workspace when the caller passed none), attn_bwd_kernel, dQ conversion.
 template <int D>
 lf_status launch_bwd(const lf_attn_desc* d, const void* q, const void* k, const void* v,
-                     const float* lse, const void* dout, const float* Dv, const float* w,
-                     const int32_t* kidx, const int32_t* kcnt, void* dq, void* dk, void* dv,
-                     void* ws, cudaStream_t st) {
+                     const void* o, const float* lse, const void* dout, const float* Dgiven,
+                     const float* w, const int32_t* kidx, const int32_t* kcnt, void* dq, void* dk,
+                     void* dv, void* ws, cudaStream_t st) {
     CUtensorMap mq, mk, mv, mdo;
     if (!make_thd_map(&mq, q, d->total_tokens, d->hq, D) ||
         !make_thd_map(&mk, k, d->total_tokens, d->hkv, D) ||
@@ -201,9 +203,12 @@ lf_status launch_bwd(const lf_attn_desc* d, const void* q, const void* k, const 
         return LF_ERR_CUDA;
     }
     const dim3 blocks(nbmax_of(d), d->hq, d->nseq);
-    lf::dq_acc_zero_kept_kernel<<<blocks, 256, 0, st>>>(d->cu_seqlens, d->total_tokens, d->max_seqlen, d->hq,
-                                                        D, d->block_q, nbmax_of(d), w, dq_acc);
+    float* Dw = Dgiven ? nullptr : reinterpret_cast<float*>(base + bwd_ws_layout(d, true).D);
+    lf::bwd_prologue_kernel<D><<<blocks, lf::kNormThreads, 0, st>>>(
+        d->cu_seqlens, d->total_tokens, d->max_seqlen, d->hq, d->block_q, nbmax_of(d), w, dq_acc,
+        static_cast<const __nv_bfloat16*>(dout), static_cast<const __nv_bfloat16*>(o), Dw);
     if (launch_status() != LF_OK) return LF_ERR_CUDA;
+    const float* Dv = Dgiven ? Dgiven : Dw;
     lf::BwdParams p{};
     p.cu_seqlens = d->cu_seqlens;
     p.T = d->total_tokens;
@@ -395,24 +400,27 @@ static lf_status block_select_impl(const lf_attn_desc* desc, const void* dout, c
         return LF_ERR_INVALID_ARG;
     }
     if (flags & ~LF_SELECT_NORMS_GIVEN) return LF_ERR_INVALID_ARG;
-    if (!dout || !o || !block_norm || !D || !tau || !block_weight || !keep || !kept_idx ||
-        !kept_cnt)
+    const bool norms_given = (flags & LF_SELECT_NORMS_GIVEN) != 0;
+    // dout is needed for the norms, o only for D
+    if ((!norms_given && !dout) || (D && (!dout || !o)) || !block_norm || !tau || !block_weight ||
+        !keep || !kept_idx || !kept_cnt)
         return LF_ERR_INVALID_ARG;
-    if (!aligned16(dout) || !aligned16(o) || !aligned16(block_norm) || !aligned16(D) ||
-        !aligned16(tau) || !aligned16(block_weight) || !aligned16(keep) || !aligned16(kept_idx) ||
-        !aligned16(kept_cnt))
-        return LF_ERR_INVALID_ARG;
+    const void* ptrs[] = {dout, o, block_norm, D, tau, block_weight, keep, kept_idx, kept_cnt};
+    for (const void* p : ptrs)
+        if (p && !aligned16(p)) return LF_ERR_INVALID_ARG;
     if ((st = pending_device_error()) != LF_OK) return st;
     if (desc->max_seqlen == 0) return LF_OK;
     const int nbmax = nbmax_of(desc);
     if ((size_t)nbmax * sizeof(double) > 200 * 1024) return LF_ERR_UNSUPPORTED;
     if ((st = prepare_device()) != LF_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const int write_norms = (flags & LF_SELECT_NORMS_GIVEN) ? 0 : 1;
-    st = desc->d == 128 ? launch_norms<128>(desc, dout, o, block_norm, D, write_norms, s)
-                        : launch_norms<64>(desc, dout, o, block_norm, D, write_norms, s);
-    if (st != LF_OK) return st;
-    const size_t smem = (size_t)nbmax * sizeof(double);
+    const int write_norms = norms_given ? 0 : 1;
+    if (write_norms || D) {
+        st = desc->d == 128 ? launch_norms<128>(desc, dout, o, block_norm, D, write_norms, s)
+                            : launch_norms<64>(desc, dout, o, block_norm, D, write_norms, s);
+        if (st != LF_OK) return st;
+    }
+    const size_t smem = (size_t)nbmax * sizeof(float);
     auto kern = rule == LF_RULE_BUDGET ? lf::select_kernel<0>
               : rule == LF_RULE_FIXED_FRACTION ? lf::select_kernel<1> : lf::select_kernel<2>;
     if (smem > 48 * 1024 &&
@@ -420,7 +428,7 @@ static lf_status block_select_impl(const lf_attn_desc* desc, const void* dout, c
             cudaSuccess)
         return LF_ERR_CUDA;
     dim3 grid(desc->hq, desc->nseq);
-    kern<<<grid, 32, smem, s>>>(desc->cu_seqlens, desc->total_tokens, desc->max_seqlen, desc->hq,
+    kern<<<grid, lf::kSelectThreads, smem, s>>>(desc->cu_seqlens, desc->total_tokens, desc->max_seqlen, desc->hq,
                                 desc->block_q, nbmax, block_norm, param, seed, step, tau,
                                 block_weight, keep, kept_idx, kept_cnt);
     return launch_status();
@@ -468,17 +476,9 @@ lf_status lf_attn_bwd(const lf_attn_desc* desc, const void* q, const void* k, co
     if (!ws || ws_bytes < bwd_ws_bytes(desc, D == nullptr)) return LF_ERR_WORKSPACE;
     if ((st = prepare_device()) != LF_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const float* Dv = D;
-    if (!Dv) {
-        float* Dw = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + bwd_ws_layout(desc, true).D);
-        st = desc->d == 128 ? launch_norms<128>(desc, dout, o, nullptr, Dw, 0, s)
-                            : launch_norms<64>(desc, dout, o, nullptr, Dw, 0, s);
-        if (st != LF_OK) return st;
-        Dv = Dw;
-    }
-    return desc->d == 128 ? launch_bwd<128>(desc, q, k, v, lse, dout, Dv, block_weight, kept_idx,
+    return desc->d == 128 ? launch_bwd<128>(desc, q, k, v, o, lse, dout, D, block_weight, kept_idx,
                                             kept_cnt, dq, dk, dv, ws, s)
-                          : launch_bwd<64>(desc, q, k, v, lse, dout, Dv, block_weight, kept_idx,
+                          : launch_bwd<64>(desc, q, k, v, o, lse, dout, D, block_weight, kept_idx,
                                            kept_cnt, dq, dk, dv, ws, s);
 }
 
@@ -506,18 +506,10 @@ lf_status lf_attn_bwd_static_ws(const lf_attn_desc* desc, const void* q, const v
     st = static_ws_address(&ws);
     if (st != LF_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    const float* Dv = D;
-    if (!Dv) {
-        float* Dw = reinterpret_cast<float*>(static_cast<uint8_t*>(ws) + bwd_ws_layout(desc, true).D);
-        st = desc->d == 128 ? launch_norms<128>(desc, dout, o, nullptr, Dw, 0, s)
-                            : launch_norms<64>(desc, dout, o, nullptr, Dw, 0, s);
-        if (st != LF_OK) return st;
-        Dv = Dw;
-    }
-    // launch_bwd clears the accumulators (cudaMemsetAsync) before the kernel
-    return desc->d == 128 ? launch_bwd<128>(desc, q, k, v, lse, dout, Dv, block_weight, kept_idx,
+    // launch_bwd clears the accumulators it uses before the kernel
+    return desc->d == 128 ? launch_bwd<128>(desc, q, k, v, o, lse, dout, D, block_weight, kept_idx,
                                             kept_cnt, dq, dk, dv, ws, s)
-                          : launch_bwd<64>(desc, q, k, v, lse, dout, Dv, block_weight, kept_idx,
+                          : launch_bwd<64>(desc, q, k, v, o, lse, dout, D, block_weight, kept_idx,
                                            kept_cnt, dq, dk, dv, ws, s);
 }
 

@@ -43,3 +43,22 @@ def rel_fro(a, b):
 def nb_per_seq(w):
     cu = w.cu_seqlens()
     return ((np.diff(cu) + w.block - 1) // w.block).astype(np.int32)
+
+
+def bf16_half_ulp(x):
+    """Half the spacing of bf16 numbers at |x| (8 significant bits): the largest
+    error the rounding of an exact value to the bf16 output format can add."""
+    a = np.abs(np.asarray(x, dtype=np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
+    return np.exp2(e - 8)
+
+
+def o_within(o, o_ref, tol):
+    """O is stored in bf16: the kernel's value may differ from the exact one by `tol`
+    (the stated max-abs tolerance) before its rounding to bf16, plus that rounding.
+    Returns (ok, worst excess, |o_ref| at the worst element) for the message."""
+    o = np.asarray(o, dtype=np.float64)
+    o_ref = np.asarray(o_ref, dtype=np.float64)
+    excess = np.abs(o - o_ref) - (tol + bf16_half_ulp(o_ref))
+    i = int(np.argmax(excess))
+    return bool(excess.flat[i] <= 0), float(excess.flat[i]), float(np.abs(o_ref).flat[i])

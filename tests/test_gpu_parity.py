@@ -3,8 +3,9 @@ same seeded bf16 inputs.
 
 Tolerances (fp32 accumulation of bf16 inputs on the GPU, fp64 in the oracle):
 keep masks, weights, tau and kept lists bit-exact given the same norm vector;
-block norms 1e-5 relative; O 1e-2 max-abs; LSE 1e-3 abs; dQ/dK/dV 1e-2
-relative Frobenius.
+block norms 1e-5 relative; O 1e-2 max-abs before its rounding to the bf16 output
+(so 1e-2 plus half a bf16 ulp of the exact value: for |O| >= 4 the rounding alone
+can exceed 1e-2); LSE 1e-3 abs; dQ/dK/dV 1e-2 relative Frobenius.
 """
 import math
 
@@ -15,7 +16,7 @@ import torch
 import block_sparse_attention_dense_b200 as lf
 import oracle
 import synthetic
-from _helpers import desc_for, nb_per_seq, rel_fro, run_step, to_dev
+from _helpers import desc_for, nb_per_seq, o_within, rel_fro, run_step, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -58,7 +59,7 @@ def test_forward_matches_oracle(w):
     o_ref, lse_ref = oracle.attn_fwd(w.cu_seqlens(), inp["q"], inp["k"], inp["v"], w.scale, w.causal)
     o = _cpu(bufs.o)
     lse = _cpu(bufs.lse)
-    assert np.abs(o - o_ref).max() < O_TOL
+    assert o_within(o, o_ref, O_TOL)[0], o_within(o, o_ref, O_TOL)
     assert np.abs(lse - lse_ref).max() < LSE_TOL
 
 
@@ -237,7 +238,7 @@ def test_noncausal_keys_of_the_next_segment_stay_out(block):
     desc, dev, bufs = run_step(w, inp)
     cu = w.cu_seqlens()
     o_ref, lse_ref = oracle.attn_fwd(cu, inp["q"], inp["k"], inp["v"], w.scale, w.causal)
-    assert np.abs(_cpu(bufs.o) - o_ref).max() < O_TOL
+    assert o_within(_cpu(bufs.o), o_ref, O_TOL)[0], o_within(_cpu(bufs.o), o_ref, O_TOL)
     dq_ref, dk_ref, dv_ref = oracle.attn_bwd(cu, inp["q"], inp["k"], inp["v"], inp["dout"],
                                              w.scale, w.block, None, w.causal)
     for got, ref in ((bufs.dq, dq_ref), (bufs.dk, dk_ref), (bufs.dv, dv_ref)):
@@ -333,7 +334,7 @@ def test_full_size_sampled_parity(w, kv_tile):
     o_ref, lse_ref = oracle.attn_fwd_rows(cu, inp["q"], inp["k"], inp["v"], w.scale, rows, heads)
     o = _cpu(bufs.o)[rows, heads]
     lse = _cpu(bufs.lse)[heads, rows]
-    assert np.abs(o - o_ref).max() < O_TOL
+    assert o_within(o, o_ref, O_TOL)[0], o_within(o, o_ref, O_TOL)
     assert np.abs(lse - lse_ref).max() < LSE_TOL
     # backward: dQ at sampled rows of kept blocks, zero at dropped blocks; dK/dV at
     # sampled rows of one KV tile (see _kv_tile_rows)
@@ -384,7 +385,7 @@ def test_gqa_mid_full_oracle():
     cu = w.cu_seqlens()
     nb = nb_per_seq(w)
     o_ref, lse_ref = oracle.attn_fwd(cu, inp["q"], inp["k"], inp["v"], w.scale, w.causal)
-    assert np.abs(_cpu(bufs.o) - o_ref).max() < O_TOL
+    assert o_within(_cpu(bufs.o), o_ref, O_TOL)[0], o_within(_cpu(bufs.o), o_ref, O_TOL)
     assert np.abs(_cpu(bufs.lse) - lse_ref).max() < LSE_TOL
     m_ref = oracle.block_norms(cu, inp["dout"], w.block, w.nbmax)
     m = _cpu(bufs.norm)
