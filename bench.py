@@ -238,11 +238,12 @@ def ClockSampler(device_index: int):
 # CPU oracle sample (the cpu_baseline and the reference arm)
 # ---------------------------------------------------------------------------
 def kernels_per_step(w: synthetic.Workload) -> int:
-    """This library's kernels in one step: forward; norms and selection; dQ
-    zeroing, backward and dQ conversion; plus the dK/dV conversions when the
-    backward's CTAs cannot hold a whole query group (group size not 1, 2 or 4)."""
+    """This library's kernels in one step: forward; norms and selection; the
+    backward's prologue (dQ accumulator rows, D), the backward and the dQ
+    conversion; plus the dK/dV conversions when one backward CTA cannot hold the
+    whole query group (more than 32 query heads per KV head)."""
     group = w.hq // w.hkv
-    return 6 + (0 if group in (1, 2, 4) else 2)
+    return 6 + (0 if group <= 32 else 2)
 
 
 def oracle_sample(w: synthetic.Workload, inp, prefix: int, seed=0, step=0):

@@ -185,11 +185,13 @@ lf_status launch_bwd(const lf_attn_desc* d, const void* q, const void* k, const 
     if (!make_acc_map(&mdvacc, dv_acc, d->total_tokens, d->hkv, D) ||
         !make_acc_map(&mdkacc, dk_acc, d->total_tokens, d->hkv, D))
         return LF_ERR_CUDA;
-    // up to four query heads of one KV head per CTA (half or a quarter of the CTAs pay
-    // the start and finish); with the whole group in one CTA, dK/dV are final in TMEM
-    // and go straight to the bf16 outputs, otherwise through fp32 accumulators
+    // one CTA per KV tile walks the whole query group of its KV head (up to
+    // kMaxHeadsPerCta heads): dK/dV are then final in TMEM and go straight to the bf16
+    // outputs, with no atomics; a larger group is split over CTAs (the largest divisor
+    // of the group within the limit) whose dK/dV tiles meet in fp32 accumulators
     const int group = d->hq / d->hkv;
-    const int heads_per_cta = group % 4 == 0 ? 4 : group % 2 == 0 ? 2 : 1;
+    int heads_per_cta = group;
+    while (heads_per_cta > lf::kMaxHeadsPerCta || group % heads_per_cta != 0) --heads_per_cta;
     const bool kv_direct = heads_per_cta == group;
     // the outputs (direct) or the dK/dV accumulators zeroed whole: rows no CTA writes
     // (no kept block reaches them, or outside every segment) read as 0; the dQ
@@ -268,6 +270,17 @@ __global__ void watchdog_selftest_kernel(long long limit) {
     if (threadIdx.x == 0) (void)mbar_wait(&bar, 0, 99, limit);
     __syncthreads();
 }
+// Enqueued at the end of every call that launches kernels: copies the failure flag,
+// once set, into the host-mapped page, so that the next call sees it without a
+// synchronization.
+__global__ void mirror_error_kernel() {
+    const int e = *reinterpret_cast<volatile int*>(&g_device_error);
+    int* m = g_error_mirror;
+    if (e != 0 && m) {
+        *reinterpret_cast<volatile int*>(m) = e;
+        __threadfence_system();
+    }
+}
 }  // namespace lf
 
 // Scratch of lf_attn_bwd_static_ws: one array per device, loaded with the
@@ -332,6 +345,13 @@ lf_status prepare_device() {
     return LF_OK;
 }
 
+// The call's kernels, then the flag's copy to the host page (stream order).
+lf_status mirror_after(lf_status launched, cudaStream_t s) {
+    if (launched != LF_OK) return launched;
+    lf::mirror_error_kernel<<<1, 1, 0, s>>>();
+    return launch_status();
+}
+
 lf_status status_of_device_code(int code) {
     if (code == 0) return LF_OK;
     return (code & 0xff) == lf::kErrTimeout ? LF_ERR_TIMEOUT : LF_ERR_INVALID_ARG;
@@ -381,8 +401,8 @@ lf_status lf_attn_fwd(const lf_attn_desc* desc, const void* q, const void* k, co
     if (desc->total_tokens == 0 || desc->max_seqlen == 0) return LF_OK;
     if ((st = prepare_device()) != LF_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    return desc->d == 128 ? launch_fwd<128>(desc, q, k, v, o, lse, s)
-                          : launch_fwd<64>(desc, q, k, v, o, lse, s);
+    return mirror_after(desc->d == 128 ? launch_fwd<128>(desc, q, k, v, o, lse, s)
+                                       : launch_fwd<64>(desc, q, k, v, o, lse, s), s);
 }
 
 static lf_status block_select_impl(const lf_attn_desc* desc, const void* dout, const void* o,
@@ -431,7 +451,7 @@ static lf_status block_select_impl(const lf_attn_desc* desc, const void* dout, c
     kern<<<grid, lf::kSelectThreads, smem, s>>>(desc->cu_seqlens, desc->total_tokens, desc->max_seqlen, desc->hq,
                                 desc->block_q, nbmax, block_norm, param, seed, step, tau,
                                 block_weight, keep, kept_idx, kept_cnt);
-    return launch_status();
+    return mirror_after(launch_status(), s);
 }
 
 lf_status lf_block_select(const lf_attn_desc* desc, const void* dout, const void* o, double delta,
@@ -476,10 +496,11 @@ lf_status lf_attn_bwd(const lf_attn_desc* desc, const void* q, const void* k, co
     if (!ws || ws_bytes < bwd_ws_bytes(desc, D == nullptr)) return LF_ERR_WORKSPACE;
     if ((st = prepare_device()) != LF_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    return desc->d == 128 ? launch_bwd<128>(desc, q, k, v, o, lse, dout, D, block_weight, kept_idx,
-                                            kept_cnt, dq, dk, dv, ws, s)
-                          : launch_bwd<64>(desc, q, k, v, o, lse, dout, D, block_weight, kept_idx,
-                                           kept_cnt, dq, dk, dv, ws, s);
+    return mirror_after(desc->d == 128 ? launch_bwd<128>(desc, q, k, v, o, lse, dout, D, block_weight,
+                                                         kept_idx, kept_cnt, dq, dk, dv, ws, s)
+                                       : launch_bwd<64>(desc, q, k, v, o, lse, dout, D, block_weight,
+                                                        kept_idx, kept_cnt, dq, dk, dv, ws, s),
+                        s);
 }
 
 lf_status lf_attn_bwd_static_ws(const lf_attn_desc* desc, const void* q, const void* k,
@@ -507,10 +528,11 @@ lf_status lf_attn_bwd_static_ws(const lf_attn_desc* desc, const void* q, const v
     if (st != LF_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     // launch_bwd clears the accumulators it uses before the kernel
-    return desc->d == 128 ? launch_bwd<128>(desc, q, k, v, o, lse, dout, D, block_weight, kept_idx,
-                                            kept_cnt, dq, dk, dv, ws, s)
-                          : launch_bwd<64>(desc, q, k, v, o, lse, dout, D, block_weight, kept_idx,
-                                           kept_cnt, dq, dk, dv, ws, s);
+    return mirror_after(desc->d == 128 ? launch_bwd<128>(desc, q, k, v, o, lse, dout, D, block_weight,
+                                                         kept_idx, kept_cnt, dq, dk, dv, ws, s)
+                                       : launch_bwd<64>(desc, q, k, v, o, lse, dout, D, block_weight,
+                                                        kept_idx, kept_cnt, dq, dk, dv, ws, s),
+                        s);
 }
 
 lf_status lf_watchdog_selftest(uint32_t limit_log2, lf_stream_t stream) {
@@ -518,9 +540,9 @@ lf_status lf_watchdog_selftest(uint32_t limit_log2, lf_stream_t stream) {
     lf_status st = pending_device_error();
     if (st != LF_OK) return st;
     if ((st = prepare_device()) != LF_OK) return st;
-    lf::watchdog_selftest_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-        1ll << limit_log2);
-    return launch_status();
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    lf::watchdog_selftest_kernel<<<1, 32, 0, s>>>(1ll << limit_log2);
+    return mirror_after(launch_status(), s);
 }
 
 lf_status lf_sync_status(lf_stream_t stream) {

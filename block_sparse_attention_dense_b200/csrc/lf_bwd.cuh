@@ -19,9 +19,9 @@
 //   tcgen05 (SS): S^T  = K_j Q_h^T,  dP^T = V_j dO_h^T        (TMEM, fp32)
 //   element-wise: P = exp2(S*scale*log2e - LSE*log2e), dS = P (dP - D), both
 //                 times the block weight; P^T and dS^T rounded to bf16 back
-//                 into TMEM (over S^T / dP^T) and dS^T into shared memory
+//                 into TMEM (both over S^T) and dS^T into shared memory
+//   tcgen05 (SS): dQ_h^T = K_j^T dS^T_h       (TMEM, over dP^T; lanes = d)
 //   tcgen05 (TS): dV_j += P^T dO_h, dK_j += dS^T Q_h   (A from TMEM)
-//   tcgen05 (SS): dQ_h^T = K_j^T dS^T_h                  (TMEM, lanes = d)
 //   dQ drain:     lane d adds column q of dQ_h^T into the fp32 accumulator;
 //                 a warp's 32 lanes hit 32 consecutive floats of one row.
 // Roles (512 threads): warp 0 TMA producer and work list, warps 1 and 2 MMA
@@ -30,9 +30,11 @@
 // each half (+ the dV and the dK epilogue respectively): thread = KV row = TMEM
 // lane; warps 8-11 dQ drain (thread = head-dim index = TMEM lane).
 //
-// Tensor memory (512 columns): dV [0,128) dK [128,256); half 0: S^T/P^T/dQ^T
-// [256,320), dP^T/dS^T [320,384); half 1: [384,448), [448,512).  Reuse of a
-// region by a later MMA relies on tcgen05.mma executing in issue order.
+// Tensor memory (512 columns): dV [0,128) dK [128,256); half 0: S^T [256,320)
+// (after the element-wise pass: P^T in its first 32 columns, dS^T in the next 32,
+// both bf16 packed two per column), dP^T then dQ^T [320,384); half 1: [384,448),
+// [448,512).  Reuse of a region by a later MMA relies on tcgen05.mma executing in
+// issue order.
 #pragma once
 
 #include "lf_device.cuh"
@@ -42,7 +44,7 @@ namespace lf {
 struct BwdParams {
     const int32_t* cu_seqlens;
     int T, hq, hkv, causal, block_q, nbmax, max_seqlen;
-    int heads_per_cta;         // 1, 2 or 4 query heads of one KV head per CTA
+    int heads_per_cta;         // query heads of one KV head per CTA (<= kMaxHeadsPerCta)
     float scale;               // softmax_scale
     float scale_log2;          // softmax_scale * log2(e)
     const float* lse;          // [hq][T], natural log
@@ -61,6 +63,7 @@ struct BwdParams {
 };
 
 constexpr uint32_t kAccBox = 128 * 32 * 4;   // one staged 32-column fp32 box of a KV tile
+constexpr int kMaxHeadsPerCta = 32;           // query heads one backward CTA can walk
 
 template <int D>
 struct BwdSmem {
@@ -73,7 +76,8 @@ struct BwdSmem {
     static constexpr uint32_t kDS = kQdo + 4 * kTile;          // two halves
     static constexpr uint32_t kVec = kDS + 2 * kHalfDS;        // lse*log2e [128], D [128]
     static constexpr uint32_t kBars = kVec + 2 * 128 * 4;
-    static constexpr uint32_t kBytes = kBars + 256;
+    static constexpr uint32_t kHeads = kBars + 256;            // int2 per query head of the CTA
+    static constexpr uint32_t kBytes = kHeads + kMaxHeadsPerCta * 8;
     static constexpr uint32_t kAlloc = kBytes + 1024;
 };
 
@@ -107,49 +111,58 @@ __device__ __forceinline__ int lower_bound_warp(const int32_t* list, int cnt, in
     return lo;
 }
 
-// Walks the kept query tiles of heads g*G .. g*G+G-1 (G <= 4) of one segment in
-// ascending order of (head, tile).  init() is called by whole warps, converged: it
-// finds every head's first kept block >= first_block with the warp-parallel search,
-// so that later steps (by any single thread) only read the lists forward.
+// Before the walk, the warps of the CTA find, head by head (warp w takes heads w,
+// w + 16, ...), each head's first kept block at or after the CTA's first query tile
+// with the warp-parallel search, and store (position, count) in shared memory; the
+// return value says whether that head has any tile to visit (the same on every lane).
+__device__ __forceinline__ bool find_head_starts(const BwdParams& p, int G, int g, int s, int jt,
+                                                 int len, int2* heads) {
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int first_block = p.causal ? (jt * 128) / p.block_q : 0;
+    const int nb = (len + p.block_q - 1) / p.block_q;
+    bool any = false;
+    for (int hh = warp; hh < G; hh += kBwdThreads / 32) {
+        const int h = g * G + hh;
+        const int32_t* l = p.kept_idx + ((size_t)s * p.hq + h) * p.nbmax;
+        const int c = min(max(p.kept_cnt[(size_t)s * p.hq + h], 0), p.nbmax);
+        const int start = first_block == 0 ? 0 : lower_bound_warp(l, c, first_block);
+        if (lane == 0) heads[hh] = make_int2(start, c);
+        if (start < c) {
+            const int b = l[start];
+            any = any || (b >= 0 && b < nb);
+        }
+    }
+    return any;
+}
+
+// Walks the kept query tiles of heads g*G .. g*G+G-1 of one segment in ascending
+// order of (head, tile), from the starts find_head_starts left in shared memory.
+// Used by one thread (the producer).
 struct KeptTileWalk {
     const int32_t* kept_idx;
-    int nbmax, hq, G, g, s, block_q, first_block, nb;
+    const int2* heads;
+    int nbmax, hq, G, g, s, block_q, nb;
     int hh, pos, cnt;
-    int starts[4], cnts[4];           // per head of the group
     const int32_t* list;
     int tile, h;
 
-    __device__ void init(const BwdParams& p, int G_, int g_, int s_, int jt, int len) {
+    __device__ void init(const BwdParams& p, const int2* heads_, int G_, int g_, int s_, int len) {
         kept_idx = p.kept_idx;
+        heads = heads_;
         nbmax = p.nbmax;
         hq = p.hq;
         G = G_;
         g = g_;
         s = s_;
         block_q = p.block_q;
-        first_block = p.causal ? (jt * 128) / p.block_q : 0;
         nb = (len + p.block_q - 1) / p.block_q;
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            starts[i] = cnts[i] = 0;
-            if (i < G) {
-                const int hi = g * G + i;
-                const int32_t* l = kept_idx + ((size_t)s * hq + hi) * nbmax;
-                const int c = min(max(p.kept_cnt[(size_t)s * hq + hi], 0), nbmax);
-                cnts[i] = c;
-                starts[i] = first_block == 0 ? 0 : lower_bound_warp(l, c, first_block);
-            }
-        }
     }
     __device__ void open_head() {
         h = g * G + hh;
         list = kept_idx + ((size_t)s * hq + h) * nbmax;
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-            if (i == hh) {
-                cnt = cnts[i];
-                pos = starts[i];
-            }
+        const int2 e = heads[hh];
+        pos = e.x;
+        cnt = e.y;
     }
     // Moves to the next tile; returns false when the walk is over.
     __device__ bool next(bool first) {
@@ -248,18 +261,19 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         tmem_alloc(tmem_slot, 512);
         tmem_relinquish();
     }
+    // every head's first kept tile for this KV tile; does the tile have any work?
+    int2* head_starts = reinterpret_cast<int2*>(smem + L::kHeads);
+    const bool has = find_head_starts(prm, prm.heads_per_cta, hgrp, s, jt, len, head_starts);
     tc_fence_before();
-    __syncthreads();
+    const bool any = __syncthreads_or(has) != 0;   // the same answer in every role
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t t_dv = tmem;
     const uint32_t t_dk = tmem + 128;
     const int kv_row0 = seg0 + jt * 128;
 
-    // Does this KV tile have any work?  (every role sees the same answer)
     KeptTileWalk walk;
-    walk.init(prm, prm.heads_per_cta, hgrp, s, jt, len);
-    const bool any = walk.next(true);
+    walk.init(prm, head_starts, prm.heads_per_cta, hgrp, s, len);
 
     constexpr uint32_t kIdescS = idesc_bf16(128, 64, 0, 0);    // S^T, dP^T halves
     constexpr uint32_t kIdescKV = idesc_bf16(128, D, 0, 1);    // dV, dK (A from TMEM, B MN-major)
@@ -278,7 +292,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 }
             }
             int n = 0;
-            bool more = any, ok = true;
+            bool more = any && walk.next(true), ok = true;
             while (more) {
                 const int st = n & 1;
                 // the stage (and, by the pipeline's order, ring slot n % 4) is free
@@ -340,31 +354,28 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             };
             const uint32_t ka = s_base + L::kK, va = s_base + L::kV;
             auto stage_q = [&](int n) { return s_base + L::kQdo + (2 * (n & 1)) * L::kTile; };
-            // S^T and dP^T of one half of pair n
-            auto issue_sdp = [&](int hf, int n) {
-                const uint32_t qa = stage_q(n), da = qa + L::kTile;
-                const uint32_t t_s = tmem + 256 + hf * 128, t_dp = t_s + 64;
+            const uint32_t t_s = tmem + 256 + hf * 128, t_dp = t_s + 64;
+            // S^T of one half of pair n (into the S^T columns)
+            auto issue_s = [&](int n) {
+                const uint32_t qa = stage_q(n);
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k)
                     mma_bf16_ss_warp(t_s, desc_kmajor(ka, k), desc_kmajor(qa + hf * 8192, k), kIdescS, k > 0);
+            };
+            // dP^T of one half of pair n (into the dP^T columns), then the commit that
+            // hands S^T and dP^T to the element-wise warps
+            auto issue_dp = [&](int n) {
+                const uint32_t da = stage_q(n) + L::kTile;
 #pragma unroll
                 for (int k = 0; k < D / 16; ++k)
                     mma_bf16_ss_warp(t_dp, desc_kmajor(va, k), desc_kmajor(da + hf * 8192, k), kIdescS, k > 0);
                 mma_commit_warp(&bar_s_full[hf]);
             };
-            // dV, dK (TS) and dQ^T (SS) of one half of pair n
-            auto issue_grads = [&](int hf, int n) {
+            // dQ^T (SS, into the dP^T columns, which the element-wise pass has read) first,
+            // so that the drain can start; then dV and dK (TS: P^T and dS^T from the S^T
+            // columns)
+            auto issue_grads = [&](int n) {
                 const uint32_t qa = stage_q(n), da = qa + L::kTile;
-                const uint32_t t_s = tmem + 256 + hf * 128, t_dp = t_s + 64;
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_bf16_ts_warp(t_dv, t_s + k * 8, desc_mnmajor(da, hf * 4 + k), kIdescKV,
-                                     (n > 0 || hf > 0 || k > 0) ? 1u : 0u);
-#pragma unroll
-                for (int k = 0; k < 4; ++k)
-                    mma_bf16_ts_warp(t_dk, t_dp + k * 8, desc_mnmajor(qa, hf * 4 + k), kIdescKV,
-                                     (n > 0 || hf > 0 || k > 0) ? 1u : 0u);
-                mma_commit_warp(&bar_qdo_empty[n & 1]);   // this half is done with the Q/dO stage
                 const uint32_t dsa = s_base + L::kDS + hf * L::kHalfDS;
 #pragma unroll
                 for (int k = 0; k < 8; ++k) {
@@ -372,19 +383,31 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     // second 64-row atom repeats the first (those lanes are unused)
                     const uint64_t adesc =
                         (D == 128) ? desc_mnmajor(ka, k) : sw128_desc(ka + k * 2048, 0, 1024);
-                    mma_bf16_ss_warp(t_s, adesc, desc_mnmajor(dsa, k), kIdescQ, k > 0);
+                    mma_bf16_ss_warp(t_dp, adesc, desc_mnmajor(dsa, k), kIdescQ, k > 0);
                 }
                 mma_commit_warp(&bar_dq_full[hf]);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16_ts_warp(t_dv, t_s + k * 8, desc_mnmajor(da, hf * 4 + k), kIdescKV,
+                                     (n > 0 || hf > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+                for (int k = 0; k < 4; ++k)
+                    mma_bf16_ts_warp(t_dk, t_s + 32 + k * 8, desc_mnmajor(qa, hf * 4 + k), kIdescKV,
+                                     (n > 0 || hf > 0 || k > 0) ? 1u : 0u);
+                mma_commit_warp(&bar_qdo_empty[n & 1]);   // this half is done with the Q/dO stage
             };
-            // Order per half: S^T/dP^T of pair n+1 goes out as soon as this half's dQ^T of
-            // pair n has been drained from TMEM.  dV and dK collect both halves in pipe
-            // order, so half 1's first gradients wait until half 0's first ones (which
-            // start the accumulators) have completed.
+            // Order per half: S^T of pair n+1 goes out right after this half's gradients of
+            // pair n (the pipe runs it after dV and dK have read P^T and dS^T from those
+            // columns); dP^T of pair n+1 as soon as the half's dQ^T of pair n has been
+            // drained from the dP^T columns.  dV and dK collect both halves in pipe order,
+            // so half 1's first gradients wait until half 0's first ones (which start the
+            // accumulators) have completed.
             bool have = wait(bar_kv, 0, 33) && wait(&bar_entry[0], 0, 34);
             have = have && ring[0].h >= 0 && wait(&bar_qdo_full[0], 0, 34);
             if (have) {
                 tc_fence_after();
-                issue_sdp(hf, 0);
+                issue_s(0);
+                issue_dp(0);
             }
             for (int n = 0; have; ++n) {
                 if (!wait(&bar_entry[(n + 1) & 3], ((n + 1) >> 2) & 1, 34)) break;
@@ -392,14 +415,15 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 if (!wait(&bar_p_ready[hf], n & 1, 36)) break;
                 if (hf == 1 && n == 0 && !wait(bar_acc0, 0, 44)) break;
                 tc_fence_after();
-                issue_grads(hf, n);
+                issue_grads(n);
                 if (hf == 0 && n == 0) mma_commit_warp(bar_acc0);
                 if (!next) break;
-                if (!wait(&bar_dq_free[hf], n & 1, 35) ||
-                    !wait(&bar_qdo_full[(n + 1) & 1], ((n + 1) >> 1) & 1, 34))
-                    break;
+                if (!wait(&bar_qdo_full[(n + 1) & 1], ((n + 1) >> 1) & 1, 34)) break;
                 tc_fence_after();
-                issue_sdp(hf, n + 1);
+                issue_s(n + 1);
+                if (!wait(&bar_dq_free[hf], n & 1, 35)) break;
+                tc_fence_after();
+                issue_dp(n + 1);
             }
             mma_commit_warp(bar_done);
             // every MMA this warp issued must finish before TMEM is released
@@ -501,8 +525,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                         dk_[2 * e4] = pack_bf16(dsw[0], dsw[1]);
                         dk_[2 * e4 + 1] = pack_bf16(dsw[2], dsw[3]);
                     }
-                    tmem_st8(t_s + c * 8, pk);     // P^T, packed columns [8c, 8c+8)
-                    tmem_st8(t_dp + c * 8, dk_);   // dS^T
+                    tmem_st8(t_s + c * 8, pk);          // P^T, packed columns [8c, 8c+8)
+                    tmem_st8(t_s + 32 + c * 8, dk_);    // dS^T, packed columns [32 + 8c, ...)
                     st_shared_v4(dsa + sw128_chunk_offset(r, 2 * c), dk_[0], dk_[1], dk_[2], dk_[3]);
                     st_shared_v4(dsa + sw128_chunk_offset(r, 2 * c + 1), dk_[4], dk_[5], dk_[6], dk_[7]);
                 };
@@ -596,7 +620,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 // the MMA issuer at once; the reductions follow off its critical path
                 float v[64];
                 if (live) {
-                    const uint32_t t_q = tmem + 256 + hf * 128 + lane_off;
+                    const uint32_t t_q = tmem + 256 + hf * 128 + 64 + lane_off;   // dP^T columns
                     uint32_t a[16], b[16];
 #pragma unroll
                     for (int c = 0; c < 4; c += 2) {

@@ -16,8 +16,11 @@ namespace lf {
 // this flag and the kernel unwinds instead of hanging the GPU.
 // ---------------------------------------------------------------------------
 __device__ int g_device_error;   // 0 = fine; otherwise (site << 8) | kind
-// Host-mapped copy of the first error (or null): lets every later host call see a
-// device-side failure without synchronizing.  Set once per device by the host.
+// Host-mapped page (or null) that mirror_error_kernel copies the flag into, so that
+// later host calls see a failure without synchronizing.  Set once per device by the
+// host.  The kernels themselves only touch g_device_error: extra code at every
+// bounded wait, even on the path taken only after a failure, slowed the backward
+// kernel's loop measurably.
 __device__ int* g_error_mirror;
 
 constexpr int kErrTimeout = 1;        // a bounded wait expired
@@ -26,14 +29,7 @@ constexpr int kErrBadSegments = 2;    // cu_seqlens inconsistent with T / max_se
 constexpr long long kWaitLimitCycles = 1ll << 31;   // ~1.1 s at 1.9 GHz
 
 __device__ __forceinline__ void report_error(int site, int kind) {
-    const int code = (site << 8) | kind;
-    if (atomicCAS(&g_device_error, 0, code) == 0) {
-        int* m = g_error_mirror;
-        if (m) {
-            *reinterpret_cast<volatile int*>(m) = code;
-            __threadfence_system();
-        }
-    }
+    atomicCAS(&g_device_error, 0, (site << 8) | kind);
 }
 __device__ __forceinline__ void report_timeout(int site) { report_error(site, kErrTimeout); }
 

@@ -39,11 +39,12 @@
  *     bounded wait expired (LF_ERR_TIMEOUT), or that found cu_seqlens
  *     inconsistent with total_tokens / max_seqlen (LF_ERR_INVALID_ARG), records
  *     the failure in a device flag and returns.  The failure is reported
- *     (1) by the next call of any entry point made after the failing kernel
- *     finished: the library mirrors the flag into a page of host memory mapped
- *     into the device, so this check needs no synchronization; that call
- *     returns the code and launches nothing; every later call does the same
- *     until the failure is cleared; and (2) by lf_sync_status (alias
+ *     (1) by the next call of any entry point made after the failing call's
+ *     work finished: every call that launches work ends with a one-thread
+ *     kernel that copies the flag into a page of host memory mapped into the
+ *     device, so this check needs no synchronization; that call returns the
+ *     code and launches nothing; every later call does the same until the
+ *     failure is cleared; and (2) by lf_sync_status (alias
  *     lf_check_device_error), which synchronizes the stream, returns the code
  *     and clears it.  The flag is one per process, shared by all streams and
  *     devices: it reports a failure of any earlier call, not only of the

@@ -37,10 +37,14 @@ SMALL = [
     # GQA without the causal mask, two segments, 64-row blocks
     synthetic.Workload("gqa_noncausal", (384, 129), hq=4, hkv=2, d=64, block=64, sigma=1.5,
                        delta=0.1, causal=False),
-    # three query heads per KV head: one head per backward CTA, dK/dV through the fp32
-    # accumulators; the forward's head-in-group index with an odd group
+    # three query heads per KV head: an odd group in one backward CTA; the forward's
+    # head-in-group index with an odd group
     synthetic.Workload("gqa3_d128", (333, 200), hq=6, hkv=2, d=128, block=128, sigma=1.5,
                        delta=0.1),
+    # 40 query heads per KV head: beyond the 32 heads one backward CTA walks, so two
+    # CTAs share each KV tile and dK/dV meet in the fp32 accumulators
+    synthetic.Workload("mqa_g40_d64", (300, 170), hq=40, hkv=1, d=64, block=128, sigma=1.5,
+                       delta=0.2),
     # 60 segments: the forward's segment search takes its multi-round path (more than 32
     # segment starts) and meets empty, one-token and tile-edge lengths (127, 128, 129, 256)
     synthetic.Workload("many_segments", (0, 1, 127, 128, 129, 256, 300, 5, 64, 200) * 6, hq=2,

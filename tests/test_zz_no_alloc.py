@@ -19,13 +19,15 @@ from _helpers import rel_fro, run_step
 GRAD_TOL = 1e-2   # the backward parity tolerance of the other GPU tests
 
 
-# two and three query heads per KV head (two group sizes of the backward's CTAs), each with
-# the selection's D and with D computed by the call itself
+# two query heads per KV head (dK/dV stored by the backward's CTAs) and forty (dK/dV through
+# fp32 accumulators in the static array), each with the selection's D and with D computed
+# by the call itself
 @pytest.mark.gpu
 @pytest.mark.parametrize("D_given", [True, False], ids=["D_given", "D_computed"])
-@pytest.mark.parametrize("hq", [4, 6], ids=["group2", "group3"])
-def test_static_scratch_backward_matches_workspace_backward_twice(hq, D_given):
-    w = synthetic.Workload("no_alloc", (700, 300), hq=hq, hkv=2, d=128, block=128, sigma=1.5,
+@pytest.mark.parametrize("hq,lens", [(4, (700, 300)), (80, (300, 200))],
+                         ids=["group2", "group40"])
+def test_static_scratch_backward_matches_workspace_backward_twice(hq, lens, D_given):
+    w = synthetic.Workload("no_alloc", lens, hq=hq, hkv=2, d=128, block=128, sigma=1.5,
                            delta=0.1)
     # one full step through the ordinary entry points (caller workspace)
     desc, dev, bufs = run_step(w, synthetic.make_inputs(w), seed=2, step=3)
