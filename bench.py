@@ -240,10 +240,12 @@ def ClockSampler(device_index: int):
 def kernels_per_step(w: synthetic.Workload) -> int:
     """This library's kernels in one step: forward; norms and selection; the
     backward's prologue (dQ accumulator rows, D), the backward and the dQ
-    conversion; plus the dK/dV conversions when one backward CTA cannot hold the
-    whole query group (more than 32 query heads per KV head)."""
+    conversion; the one-thread kernel that ends each of the three calls (it copies
+    the device failure flag to the host-mapped page); plus the dK/dV conversions
+    when one backward CTA cannot hold the whole query group (more than 32 query
+    heads per KV head)."""
     group = w.hq // w.hkv
-    return 6 + (0 if group <= 32 else 2)
+    return 9 + (0 if group <= 32 else 2)
 
 
 def oracle_sample(w: synthetic.Workload, inp, prefix: int, seed=0, step=0):
@@ -541,6 +543,44 @@ def main():
 
     # ---- the dense backward (delta = 0) through the same kernels: does the backward's
     # time follow the executed fraction?  (article section "A 32 000 tokens, 5,72 fois")
+    # ---- selection telemetry beyond the workload's own delta (outside the timed regions):
+    # the speech setting's delta = 0.4 on the same gradients, and the kept fraction at
+    # causal prefixes of the sequence (a prefix is itself a complete problem, with the
+    # same per-block gradient scales), article sections "Un budget qui ne se transpose
+    # pas du texte à la parole" and "Le choix des blocs pèse plus que la quantité sautée"
+    if rule_id == 0 and w.nseq == 1 and not args.no_dense_arm:
+        extra = {}
+
+        def sel_bufs(dsc):
+            nbm = (dsc.max_seqlen + dsc.block_q - 1) // dsc.block_q
+            f32 = dict(dtype=torch.float32, device=dev)
+            return dict(norm=torch.empty(dsc.nseq, w.hq, nbm, **f32),
+                        D=torch.empty(w.hq, dsc.total_tokens, **f32),
+                        tau=torch.empty(dsc.nseq, w.hq, dtype=torch.float64, device=dev),
+                        w=torch.empty(dsc.nseq, w.hq, nbm, **f32),
+                        keep=torch.empty(dsc.nseq, w.hq, nbm, dtype=torch.uint8, device=dev),
+                        kept_idx=torch.empty(dsc.nseq, w.hq, nbm, dtype=torch.int32, device=dev),
+                        kept_cnt=torch.empty(dsc.nseq, w.hq, dtype=torch.int32, device=dev))
+
+        def run_select(dsc, dout, o, delta):
+            b = sel_bufs(dsc)
+            lf.lf_block_select(dsc, dout, o, delta, 0, 0, 0, b["norm"], b["D"], b["tau"], b["w"],
+                               b["keep"], b["kept_idx"], b["kept_cnt"])
+            nb = (dsc.total_tokens + w.block - 1) // w.block
+            return float(b["keep"][:, :, :nb].float().mean())
+
+        extra["delta_0.4_kept_fraction"] = run_select(desc, d_in["dout"], bufs.o, 0.4)
+        by_len = {}
+        for n_tok in (8192, 16384, 32768, 65536):
+            if n_tok > w.total_tokens:
+                continue
+            cu_p = torch.tensor([0, n_tok], dtype=torch.int32, device=dev)
+            dp = lf.make_desc(cu_p, n_tok, n_tok, w.hq, w.hkv, w.d, w.scale, w.causal, w.block)
+            by_len[str(n_tok)] = run_select(dp, d_in["dout"][:n_tok], bufs.o[:n_tok], w.delta)
+        extra["kept_fraction_by_length_at_delta"] = by_len
+        lf.lf_sync_status()
+        telemetry.update(extra)
+
     dense_arm = None
     if rule_id == 0 and w.delta > 0 and not args.no_dense_arm:
         K0 = max(3, K // 2)

@@ -144,7 +144,8 @@ lf_status launch_fwd(const lf_attn_desc* d, const void* q, const void* k, const 
     if (launch_regs * lf::kFwdThreads < 128 * lf::kFwdCtrlRegs + 256 * lf::kFwdSoftmaxRegs)
         return LF_ERR_UNSUPPORTED;
     // one CTA per pair of query tiles; the query heads of one KV head together, their
-    // longest pairs first (x = pair rank * group + head in group, y = KV head)
+    // longest pairs first within each segment (x = pair rank * group + head in group,
+    // y = KV head)
     // (x: pairs of query tiles over all segments, flattened; see segment_of_unit)
     const long long pair_units = ((long long)d->total_tokens + 255ll * d->nseq) >> 8;
     dim3 grid(static_cast<unsigned>(pair_units * (d->hq / d->hkv)), d->hkv, 1);

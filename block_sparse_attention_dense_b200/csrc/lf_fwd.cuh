@@ -80,8 +80,9 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
 
     // blockIdx.x = pair * G + query head within the KV head's group, the pairs of
     // 256 query rows running over all segments, segment by segment; blockIdx.y = KV
-    // head.  The G query heads that share a KV head run together, longest rows first,
-    // so their K/V stay in L2 and each group's work outlasts its heaviest CTA.
+    // head.  The G query heads that share a KV head run together, longest rows first
+    // within each segment, so their K/V stay in L2 and each group's work outlasts its
+    // heaviest CTA.
     const int G = prm.hq / prm.hkv;
     const int g = blockIdx.y;
     const int h = g * G + static_cast<int>(blockIdx.x) % G;

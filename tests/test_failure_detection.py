@@ -63,3 +63,28 @@ def test_next_call_reports_the_expired_wait_without_a_sync():
     lf.lf_attn_fwd(desc, dev["q"], dev["k"], dev["v"], marker, bufs.lse)
     lf.lf_sync_status()
     assert torch.equal(marker, bufs.o)
+
+
+@pytest.mark.gpu
+def test_bad_segment_table_is_reported_by_the_next_call():
+    """cu_seqlens that disagree with total_tokens (a segment ending past T) are found on
+    the device: the kernels skip that segment without touching its rows, and the next
+    call returns LF_ERR_INVALID_ARG until lf_sync_status clears it."""
+    lf.lf_sync_status()
+    w = synthetic.TINY
+    inp = synthetic.make_inputs(w)
+    desc, dev, bufs = run_step(w, inp)
+    bad_cu = torch.tensor([0, w.total_tokens + 64], dtype=torch.int32, device="cuda")
+    bad = lf.make_desc(bad_cu, w.total_tokens + 64, w.total_tokens, w.hq, w.hkv, w.d, w.scale,
+                       w.causal, w.block)
+    lf.lf_attn_fwd(bad, dev["q"], dev["k"], dev["v"], bufs.o, bufs.lse)
+    torch.cuda.synchronize()
+    with pytest.raises(lf.LfError) as ei:
+        lf.lf_attn_fwd(desc, dev["q"], dev["k"], dev["v"], bufs.o, bufs.lse)
+    assert ei.value.code == lf.LF_ERR_INVALID_ARG
+    with pytest.raises(lf.LfError) as ei:
+        lf.lf_sync_status()
+    assert ei.value.code == lf.LF_ERR_INVALID_ARG
+    lf.lf_sync_status()
+    _, _, again = run_step(w, inp)
+    assert torch.equal(again.o, bufs.o)
