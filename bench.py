@@ -415,6 +415,60 @@ def run_layers(args, w):
     print(json.dumps(line), flush=True)
 
 
+def measure_workload(lf, w, dev, steps=5, warmup=2):
+    """fwd / select / bwd ms (CUDA events on the launching stream, inputs resident) of
+    one synthetic workload at its own delta, with its executed and dense-equivalent
+    backward FLOPs: the other configurations of the measurement plan, reported beside
+    the headline line."""
+    stream = torch.cuda.current_stream()
+    inp = synthetic.make_inputs(w)
+    d_in = {k: v.to(dev) for k, v in inp.items() if k != "cu_seqlens"}
+    cu = inp["cu_seqlens"].to(dev)
+    desc = lf.make_desc(cu, w.max_seqlen, w.total_tokens, w.hq, w.hkv, w.d, w.scale, w.causal,
+                        w.block)
+    b = lf.Buffers(desc, device=dev)
+
+    def run(record=None):
+        ev = record or [None] * 4
+        if ev[0]: ev[0].record(stream)
+        lf.lf_attn_fwd(desc, d_in["q"], d_in["k"], d_in["v"], b.o, b.lse)
+        if ev[1]: ev[1].record(stream)
+        lf.lf_block_select(desc, d_in["dout"], b.o, w.delta, 0, 0, 0, b.norm, b.D, b.tau, b.w,
+                           b.keep, b.kept_idx, b.kept_cnt)
+        if ev[2]: ev[2].record(stream)
+        lf.lf_attn_bwd(desc, d_in["q"], d_in["k"], d_in["v"], b.o, b.lse, d_in["dout"], b.D, b.w,
+                       b.kept_idx, b.kept_cnt, b.dq, b.dk, b.dv, b.ws)
+        if ev[3]: ev[3].record(stream)
+
+    for _ in range(warmup):
+        run()
+    torch.cuda.synchronize()
+    # smaller workloads fit in L2: a 256 MB write before every timed step (outside the
+    # phase events) leaves each step to start from HBM
+    flush = torch.empty(64 << 20, dtype=torch.float32, device=dev)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for e in evs:
+        flush.zero_()
+        run(e)
+    torch.cuda.synchronize()
+    del flush
+    lf.lf_sync_status()
+    fwd_ms = sum(e[0].elapsed_time(e[1]) for e in evs) / steps
+    sel_ms = sum(e[1].elapsed_time(e[2]) for e in evs) / steps
+    bwd_ms = sum(e[2].elapsed_time(e[3]) for e in evs) / steps
+    keep = b.keep.cpu().numpy()
+    fwd_fl, bwd_dense_fl, bwd_exec_fl = tile_flops(w, keep)
+    out = {"tokens": w.total_tokens, "segments": w.nseq, "delta": w.delta,
+           "fwd_ms": fwd_ms, "select_ms": sel_ms, "bwd_ms": bwd_ms,
+           "fwd_tflops": fwd_fl / (fwd_ms * 1e-3) / 1e12,
+           "bwd_tflops_executed": bwd_exec_fl / (bwd_ms * 1e-3) / 1e12,
+           "bwd_executed_fraction": bwd_exec_fl / bwd_dense_fl, "steps": steps,
+           "l2": "256 MB written before every timed step"}
+    del b, d_in
+    torch.cuda.empty_cache()
+    return out
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -746,6 +800,20 @@ def main():
             "sample": "oracle backward (executed tile FLOPs over its time) on the first %d tokens "
                       "of the %s workload, all %d heads; its forward and selection ran untimed"
                       % (min(args.cpu_prefix, w.seqlens[0]), w.name, w.hq)}
+    if rank == 0 and n == 1 and args.workload == "headline" and not args.no_dense_arm:
+        # the other configurations of the measurement plan, each at its own delta (the
+        # Long workload also at delta 0, the dense backward): context beside the headline
+        others = {}
+        for name, ww in (("gqa_mid", synthetic.GQA_MID),
+                         ("long_delta0", synthetic.LONG.with_(delta=0.0)),
+                         ("long_delta0.05", synthetic.LONG.with_(delta=0.05)),
+                         ("long_delta0.2", synthetic.LONG.with_(delta=0.2)),
+                         ("varlen", synthetic.VARLEN)):
+            others[name] = measure_workload(lf, ww, dev)
+        base = others["long_delta0"]["bwd_ms"]
+        for name in ("long_delta0.05", "long_delta0.2"):
+            others[name]["bwd_time_vs_delta0"] = others[name]["bwd_ms"] / base
+        line["other_workloads"] = others
     if rank == 0:
         print(json.dumps(line), flush=True)
     if dist is not None:
