@@ -78,13 +78,13 @@ BwdWs bwd_ws_layout(const lf_attn_desc* d, bool need_D) {
 }
 size_t bwd_ws_bytes(const lf_attn_desc* d, bool need_D) { return bwd_ws_layout(d, need_D).total; }
 
-// [T][H][d] bf16 -> 3-D map (d, H, T), 64 x 1 x 128 boxes, 128-byte swizzle.
-bool make_thd_map(CUtensorMap* m, const void* base, int T, int H, int D) {
+// [T][H][d] bf16 -> 3-D map (d, H, T), 64 x 1 x `rows` boxes, 128-byte swizzle.
+bool make_thd_map(CUtensorMap* m, const void* base, int T, int H, int D, int rows = 128) {
     EncodeTiledFn enc = encode_tiled();
     if (!enc) return false;
     const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)T};
     const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)H * D * 2};
-    const cuuint32_t box[3] = {64, 1, 128};
+    const cuuint32_t box[3] = {64, 1, (cuuint32_t)rows};
     const cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box,
                estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -171,11 +171,14 @@ lf_status launch_bwd(const lf_attn_desc* d, const void* q, const void* k, const 
                      const void* o, const float* lse, const void* dout, const float* Dgiven,
                      const float* w, const int32_t* kidx, const int32_t* kcnt, void* dq, void* dk,
                      void* dv, void* ws, cudaStream_t st) {
-    CUtensorMap mq, mk, mv, mdo;
+    // Q and dO also in 64-row boxes: a query tile with one live half loads only that half
+    CUtensorMap mq, mk, mv, mdo, mq64, mdo64;
     if (!make_thd_map(&mq, q, d->total_tokens, d->hq, D) ||
         !make_thd_map(&mk, k, d->total_tokens, d->hkv, D) ||
         !make_thd_map(&mv, v, d->total_tokens, d->hkv, D) ||
-        !make_thd_map(&mdo, dout, d->total_tokens, d->hq, D))
+        !make_thd_map(&mdo, dout, d->total_tokens, d->hq, D) ||
+        !make_thd_map(&mq64, q, d->total_tokens, d->hq, D, 64) ||
+        !make_thd_map(&mdo64, dout, d->total_tokens, d->hq, D, 64))
         return LF_ERR_CUDA;
     const BwdWs lay = bwd_ws_layout(d, false);
     uint8_t* base = static_cast<uint8_t*>(ws);
@@ -234,11 +237,12 @@ lf_status launch_bwd(const lf_attn_desc* d, const void* q, const void* k, const 
     p.kept_cnt = kcnt;
     p.dq_acc = dq_acc;
     const uint32_t smem = lf::BwdSmem<D>::kAlloc;
-    if (cudaFuncSetAttribute(lf::attn_bwd_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
+    // 64-row selection blocks: the variant that skips a tile's dropped half
+    auto kern = d->block_q == 64 ? lf::attn_bwd_kernel<D, true> : lf::attn_bwd_kernel<D, false>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return LF_ERR_CUDA;
     dim3 grid(ntiles_of(d), d->hq / p.heads_per_cta, d->nseq);
-    lf::attn_bwd_kernel<D><<<grid, lf::kBwdThreads, smem, st>>>(mq, mk, mv, mdo, mdvacc, mdkacc, p);
+    kern<<<grid, lf::kBwdThreads, smem, st>>>(mq, mk, mv, mdo, mdvacc, mdkacc, mq64, mdo64, p);
     if (launch_status() != LF_OK) return LF_ERR_CUDA;
     // fp32 accumulators -> bf16 results (dQ and dK take the softmax scale)
     const size_t nkv8 = (size_t)d->total_tokens * d->hkv * D / 8;

@@ -30,6 +30,15 @@
 // each half (+ the dV and the dK epilogue respectively): thread = KV row = TMEM
 // lane; warps 8-11 dQ drain (thread = head-dim index = TMEM lane).
 //
+// kHalves (64-row selection blocks): a query half is one block and is live when its
+// weight is non-zero; a dropped block's half is neither loaded (a tile with one live
+// half loads Q and dO in 64-row boxes) nor computed, and a half past the segment's end
+// is skipped the same way.  Every role counts a half's barrier phases by its live
+// pairs, and dV and dK start from zeros stored in TMEM, so the first gradient MMA of
+// either half may come first.  With 128-row blocks both halves of a tile carry the
+// same block's weight, and the kernel keeps one phase per pair (the skipping
+// variant's bookkeeping cost about 4 % there, A/B on one GPU).
+//
 // Tensor memory (512 columns): dV [0,128) dK [128,256); half 0: S^T [256,320)
 // (after the element-wise pass: P^T in its first 32 columns, dS^T in the next 32,
 // both bf16 packed two per column), dP^T then dQ^T [320,384); half 1: [384,448),
@@ -195,11 +204,12 @@ __device__ __forceinline__ float half_weight(const BwdParams& p, int s, int h, i
     return p.block_weight[((size_t)s * p.hq + h) * p.nbmax + q0 / p.block_q];
 }
 
-template <int D>
+template <int D, bool kHalves>
 __global__ void __launch_bounds__(kBwdThreads, 1)
     attn_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_dvacc, const __grid_constant__ CUtensorMap tm_dkacc,
+                    const __grid_constant__ CUtensorMap tm_q64, const __grid_constant__ CUtensorMap tm_do64,
                     BwdParams prm) {
     using L = BwdSmem<D>;
     static_assert(2 * (D / 32) * kAccBox <= 4 * L::kTile, "dK/dV staging must fit the Q/dO buffers");
@@ -220,7 +230,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 15);
     uint64_t* bar_entry = bars + 16;      // [4] work-list ring
     PairEntry* ring = reinterpret_cast<PairEntry*>(bars + 20);   // [4] x 16 B
-    uint64_t* bar_acc0 = bars + 28;       // one phase: half 0's first dV/dK MMAs completed
+    uint64_t* bar_acc0 = bars + 28;       // one phase: half 0's first dV/dK MMAs completed (!kHalves)
 
     // KV tile fastest: CTAs resident together share one query head, so its Q,
     // dO and dQ accumulator stay in L2; the lowest tiles (most work) start first
@@ -246,8 +256,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             mbar_init(&bar_dq_free[i], 128);
         }
         mbar_init(bar_done, 2);                 // one commit per MMA issuer
-        mbar_init(bar_acc0, 1);
         for (int i = 0; i < 4; ++i) mbar_init(&bar_entry[i], 1);
+        mbar_init(bar_acc0, 1);
         *abort_flag = 0;
         fence_barrier_init();
         prefetch_tensormap(&tm_q);
@@ -256,6 +266,8 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         prefetch_tensormap(&tm_do);
         prefetch_tensormap(&tm_dvacc);
         prefetch_tensormap(&tm_dkacc);
+        prefetch_tensormap(&tm_q64);
+        prefetch_tensormap(&tm_do64);
     }
     if (warp == 0) {
         tmem_alloc(tmem_slot, 512);
@@ -308,12 +320,21 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 e.w1 = half_weight(prm, s, walk.h, q0 + 64, len);
                 ring[n & 3] = e;
                 mbar_arrive(&bar_entry[n & 3]);
-                const int row = seg0 + q0;
-                mbar_arrive_expect_tx(&bar_qdo_full[st], 2 * L::kTile);
+                // Q and dO rows of the tile's live halves only: both halves in 128-row boxes,
+                // a single live half in 64-row boxes; a half whose block was dropped, or that
+                // lies past the segment's end, is not loaded
+                const bool live0 = !kHalves || e.w0 != 0.f, live1 = !kHalves || e.w1 != 0.f;
+                const uint32_t nlive = (live0 ? 1u : 0u) + (live1 ? 1u : 0u);
+                mbar_arrive_expect_tx(&bar_qdo_full[st], nlive * L::kTile);
+                const int hh = live0 ? 0 : 1;                     // the single live half
+                const CUtensorMap* mq = nlive == 2 ? &tm_q : &tm_q64;
+                const CUtensorMap* mdo = nlive == 2 ? &tm_do : &tm_do64;
+                const int row = seg0 + q0 + (nlive == 2 ? 0 : 64 * hh);
+                const uint32_t off = nlive == 2 ? 0u : hh * 8192u;
                 for (int c = 0; c < L::kPanels; ++c) {
-                    tma_load_3d(smem + L::kQdo + (2 * st) * L::kTile + c * kPanelBytes, &tm_q,
+                    tma_load_3d(smem + L::kQdo + (2 * st) * L::kTile + c * kPanelBytes + off, mq,
                                 &bar_qdo_full[st], c * 64, walk.h, row);
-                    tma_load_3d(smem + L::kQdo + (2 * st + 1) * L::kTile + c * kPanelBytes, &tm_do,
+                    tma_load_3d(smem + L::kQdo + (2 * st + 1) * L::kTile + c * kPanelBytes + off, mdo,
                                 &bar_qdo_full[st], c * 64, walk.h, row);
                 }
                 fill_parity[st] = (n >> 1) & 1;
@@ -386,44 +407,93 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                     mma_bf16_ss_warp(t_dp, adesc, desc_mnmajor(dsa, k), kIdescQ, k > 0);
                 }
                 mma_commit_warp(&bar_dq_full[hf]);
+                // kHalves: dV and dK accumulate onto TMEM the element-wise warps zeroed at
+                // the start; otherwise half 0's first ones start them
+                const uint32_t first = (kHalves || n > 0 || hf > 0) ? 1u : 0u;
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                     mma_bf16_ts_warp(t_dv, t_s + k * 8, desc_mnmajor(da, hf * 4 + k), kIdescKV,
-                                     (n > 0 || hf > 0 || k > 0) ? 1u : 0u);
+                                     (first || k > 0) ? 1u : 0u);
 #pragma unroll
                 for (int k = 0; k < 4; ++k)
                     mma_bf16_ts_warp(t_dk, t_s + 32 + k * 8, desc_mnmajor(qa, hf * 4 + k), kIdescKV,
-                                     (n > 0 || hf > 0 || k > 0) ? 1u : 0u);
+                                     (first || k > 0) ? 1u : 0u);
                 mma_commit_warp(&bar_qdo_empty[n & 1]);   // this half is done with the Q/dO stage
             };
-            // Order per half: S^T of pair n+1 goes out right after this half's gradients of
-            // pair n (the pipe runs it after dV and dK have read P^T and dS^T from those
-            // columns); dP^T of pair n+1 as soon as the half's dQ^T of pair n has been
-            // drained from the dP^T columns.  dV and dK collect both halves in pipe order,
-            // so half 1's first gradients wait until half 0's first ones (which start the
-            // accumulators) have completed.
-            bool have = wait(bar_kv, 0, 33) && wait(&bar_entry[0], 0, 34);
-            have = have && ring[0].h >= 0 && wait(&bar_qdo_full[0], 0, 34);
-            if (have) {
-                tc_fence_after();
-                issue_s(0);
-                issue_dp(0);
-            }
-            for (int n = 0; have; ++n) {
-                if (!wait(&bar_entry[(n + 1) & 3], ((n + 1) >> 2) & 1, 34)) break;
-                const bool next = ring[(n + 1) & 3].h >= 0;
-                if (!wait(&bar_p_ready[hf], n & 1, 36)) break;
-                if (hf == 1 && n == 0 && !wait(bar_acc0, 0, 44)) break;
-                tc_fence_after();
-                issue_grads(n);
-                if (hf == 0 && n == 0) mma_commit_warp(bar_acc0);
-                if (!next) break;
-                if (!wait(&bar_qdo_full[(n + 1) & 1], ((n + 1) >> 1) & 1, 34)) break;
-                tc_fence_after();
-                issue_s(n + 1);
-                if (!wait(&bar_dq_free[hf], n & 1, 35)) break;
-                tc_fence_after();
-                issue_dp(n + 1);
+            // Order per half: S^T of the next pair goes out right after this half's gradients
+            // (the pipe runs it after dV and dK have read P^T and dS^T from those columns);
+            // its dP^T as soon as the half's last dQ^T has been drained from the dP^T
+            // columns.  A pair whose half is not live (its 64-row block dropped, or past the
+            // segment's end) is skipped by every role of that half: the half's barriers
+            // count live pairs (kg), and only the Q/dO stage is released for it.
+            if constexpr (kHalves) {
+                auto live = [&](const PairEntry& x) { return (hf ? x.w1 : x.w0) != 0.f; };
+                int kg = 0;                  // this half's live pairs whose gradients are issued
+                bool pending_free = false;   // the last dQ^T still occupies the dP^T columns
+                bool have = wait(bar_kv, 0, 33) && wait(&bar_entry[0], 0, 34);
+                PairEntry cur = ring[0];
+                have = have && cur.h >= 0;
+                if (have && live(cur)) {
+                    have = wait(&bar_qdo_full[0], 0, 34);
+                    if (have) {
+                        tc_fence_after();
+                        issue_s(0);
+                        issue_dp(0);
+                    }
+                }
+                for (int n = 0; have; ++n) {
+                    if (!wait(&bar_entry[(n + 1) & 3], ((n + 1) >> 2) & 1, 34)) break;
+                    const PairEntry nxt = ring[(n + 1) & 3];
+                    if (live(cur)) {
+                        if (!wait(&bar_p_ready[hf], kg & 1, 36)) break;
+                        tc_fence_after();
+                        issue_grads(n);
+                        ++kg;
+                        pending_free = true;
+                    } else {
+                        mma_commit_warp(&bar_qdo_empty[n & 1]);   // nothing of this half reads the stage
+                    }
+                    if (nxt.h < 0) break;
+                    if (live(nxt)) {
+                        if (!wait(&bar_qdo_full[(n + 1) & 1], ((n + 1) >> 1) & 1, 34)) break;
+                        tc_fence_after();
+                        issue_s(n + 1);
+                        if (pending_free) {
+                            if (!wait(&bar_dq_free[hf], (kg - 1) & 1, 35)) break;
+                            pending_free = false;
+                            tc_fence_after();
+                        }
+                        issue_dp(n + 1);
+                    }
+                    cur = nxt;
+                }
+            } else {
+                // one phase per pair: dV and dK collect both halves in pipe order, so half
+                // 1's first gradients wait until half 0's first ones (which start the
+                // accumulators) have completed
+                bool have = wait(bar_kv, 0, 33) && wait(&bar_entry[0], 0, 34);
+                have = have && ring[0].h >= 0 && wait(&bar_qdo_full[0], 0, 34);
+                if (have) {
+                    tc_fence_after();
+                    issue_s(0);
+                    issue_dp(0);
+                }
+                for (int n = 0; have; ++n) {
+                    if (!wait(&bar_entry[(n + 1) & 3], ((n + 1) >> 2) & 1, 34)) break;
+                    const bool next = ring[(n + 1) & 3].h >= 0;
+                    if (!wait(&bar_p_ready[hf], n & 1, 36)) break;
+                    if (hf == 1 && n == 0 && !wait(bar_acc0, 0, 44)) break;
+                    tc_fence_after();
+                    issue_grads(n);
+                    if (hf == 0 && n == 0) mma_commit_warp(bar_acc0);
+                    if (!next) break;
+                    if (!wait(&bar_qdo_full[(n + 1) & 1], ((n + 1) >> 1) & 1, 34)) break;
+                    tc_fence_after();
+                    issue_s(n + 1);
+                    if (!wait(&bar_dq_free[hf], n & 1, 35)) break;
+                    tc_fence_after();
+                    issue_dp(n + 1);
+                }
             }
             mma_commit_warp(bar_done);
             // every MMA this warp issued must finish before TMEM is released
@@ -442,7 +512,23 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         // its exponent is not bounded by this query's LSE and must not reach the products)
         const int kv_cmp = !kv_valid ? 0x7fffffff : (prm.causal ? kv_local : (int)0x80000000);
         int n = 0;
+        // parity of each half's live pairs processed (bit hf: the half's barrier phase);
+        // bits of one register rather than an array indexed by the half loop, which would
+        // live in local memory
+        uint32_t ke = 0;
         bool more = any, failed = false;
+        if (kHalves && any) {
+            // dV (warpgroup 0) and dK (warpgroup 1) start from zero in TMEM, so that every
+            // gradient MMA accumulates, whichever half and pair comes first; the stores are
+            // complete before this warpgroup's first p_ready arrival
+            const uint32_t t_acc = (wg ? t_dk : t_dv) + lane_off;
+            float z[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) z[i] = 0.f;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) tmem_st32(t_acc + c * 32, z);
+            tmem_wait_st();
+        }
         for (;;) {
             // uniform decision of both warpgroups; also: all are done with the old vectors
             if (named_bar_or(1, 256, !more || failed)) break;
@@ -470,9 +556,11 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             named_bar_sync(2, 256);
             for (int hf = 0; hf < 2; ++hf) {
                 const float w = hf ? e.w1 : e.w0;
+                if (kHalves && w == 0.f) continue;   // not live: nothing was loaded or computed for it
                 const uint32_t t_s = tmem + 256 + hf * 128 + lane_off, t_dp = t_s + 64;
                 const uint32_t dsa = s_base + L::kDS + hf * L::kHalfDS;
-                const bool got = mbar_wait_or_abort(&bar_s_full[hf], n & 1, 38, abort_flag);
+                const uint32_t par = kHalves ? (ke >> hf) & 1u : static_cast<uint32_t>(n & 1);
+                const bool got = mbar_wait_or_abort(&bar_s_full[hf], par, 38, abort_flag);
                 const bool ok = __all_sync(0xffffffffu, got);
                 // this warpgroup's two 16-column chunks of S^T and dP^T
                 uint32_t sa[16], da[16], sb[16], db[16];
@@ -536,6 +624,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
                 fence_proxy_async_smem();
                 tc_fence_before();
                 mbar_arrive(&bar_p_ready[hf]);
+                ke ^= 1u << hf;
             }
             if (!failed) ++n;
         }
@@ -602,6 +691,7 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
         const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
         const bool lane_used = (warp & 3) * 32 < D;       // d = 64: warps 10, 11 idle
         int n = 0;
+        uint32_t kd = 0;      // parity of each half's live pairs drained (bit hf)
         bool more = any;
         while (more) {
             const bool got_e = mbar_wait_or_abort(&bar_entry[n & 3], (n >> 2) & 1, 42, abort_flag);
@@ -611,11 +701,14 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
             const int q0 = e.tile * 128;
             bool ok = true;
             for (int hf = 0; hf < 2; ++hf) {
-                const bool got = mbar_wait_or_abort(&bar_dq_full[hf], n & 1, 40, abort_flag);
+                if (kHalves && (hf ? e.w1 : e.w0) == 0.f) continue;   // not live: no dQ^T for this half
+                const uint32_t par = kHalves ? (kd >> hf) & 1u : static_cast<uint32_t>(n & 1);
+                const bool got = mbar_wait_or_abort(&bar_dq_full[hf], par, 40, abort_flag);
                 if (!__all_sync(0xffffffffu, got)) { ok = false; break; }
+                kd ^= 1u << hf;
                 tc_fence_after();
                 const int qh = q0 + hf * 64;
-                const bool live = lane_used && qh < len && (hf ? e.w1 : e.w0) != 0.f;
+                const bool live = lane_used && qh < len && (kHalves || (hf ? e.w1 : e.w0) != 0.f);
                 // copy the half's dQ^T to registers and hand its TMEM columns back to
                 // the MMA issuer at once; the reductions follow off its critical path
                 float v[64];

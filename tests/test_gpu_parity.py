@@ -496,3 +496,37 @@ def test_backward_with_topk_and_fixed_fraction_weights():
         assert rel_fro(_cpu(bufs.dq), dq_ref) < GRAD_TOL
         assert rel_fro(_cpu(bufs.dk), dk_ref) < GRAD_TOL
         assert rel_fro(_cpu(bufs.dv), dv_ref) < GRAD_TOL
+
+
+@pytest.mark.parametrize("w", [SMALL[0], SMALL[4], SMALL[1]], ids=lambda w: w.name)
+def test_dropped_blocks_are_never_read(w):
+    """Dropped tiles are never loaded or computed (article section "Un budget sur la
+    masse de gradient ..."): after the selection, the Q and dO rows of every dropped
+    block are overwritten with NaN; a backward that loaded or multiplied any of them
+    (even by a zero weight) would return NaN.  With 64-row blocks this covers the
+    dropped half of a 128-row tile whose other half is kept."""
+    inp = synthetic.make_inputs(w)
+    desc, dev, bufs = run_step(w, inp, seed=3, step=1)
+    cu = w.cu_seqlens()
+    nb = nb_per_seq(w)
+    keep = bufs.keep.cpu().numpy()
+    q_bad, do_bad = dev["q"].clone(), dev["dout"].clone()
+    dropped = 0
+    for s in range(w.nseq):
+        for h in range(w.hq):
+            for b in range(int(nb[s])):
+                if keep[s, h, b] == 0:
+                    r0 = int(cu[s]) + b * w.block
+                    r1 = min(r0 + w.block, int(cu[s + 1]))
+                    q_bad[r0:r1, h] = float("nan")
+                    do_bad[r0:r1, h] = float("nan")
+                    dropped += 1
+    assert dropped > 0
+    out = {k: torch.empty_like(getattr(bufs, k)) for k in ("dq", "dk", "dv")}
+    lf.lf_attn_bwd(desc, q_bad, dev["k"], dev["v"], bufs.o, bufs.lse, do_bad, bufs.D, bufs.w,
+                   bufs.kept_idx, bufs.kept_cnt, out["dq"], out["dk"], out["dv"], bufs.ws)
+    lf.lf_sync_status()
+    for k in ("dq", "dk", "dv"):
+        got = out[k].float().cpu()
+        assert torch.isfinite(got).all(), k
+        assert rel_fro(got, getattr(bufs, k).float().cpu()) < 1e-5, k
