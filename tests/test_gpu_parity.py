@@ -45,6 +45,10 @@ SMALL = [
     # CTAs share each KV tile and dK/dV meet in the fp32 accumulators
     synthetic.Workload("mqa_g40_d64", (300, 170), hq=40, hkv=1, d=64, block=128, sigma=1.5,
                        delta=0.2),
+    # the same split group with 64-row blocks: the half-skipping backward on the
+    # accumulator path
+    synthetic.Workload("mqa_g40_blk64", (200, 90), hq=40, hkv=1, d=64, block=64, sigma=2.0,
+                       delta=0.3),
     # 60 segments: the forward's segment search takes its multi-round path (more than 32
     # segment starts) and meets empty, one-token and tile-edge lengths (127, 128, 129, 256)
     synthetic.Workload("many_segments", (0, 1, 127, 128, 129, 256, 300, 5, 64, 200) * 6, hq=2,
