@@ -121,7 +121,10 @@ lf_status lf_attn_fwd(const lf_attn_desc* desc, const void* q, const void* k, co
  *   block_weight[s][h][i] = (float)(1 / p_i) if kept else 0;
  *   keep (uint8), kept_idx (int32, ascending kept block indices, -1 padded),
  *   kept_cnt[s][h] (int32).
- *   delta must lie in [0, 1).  dout and o are [T][hq][d] bf16. */
+ *   delta must lie in [0, 1).  dout and o are [T][hq][d] bf16.  D may be NULL: the
+ *   norm pass then reads dout only (o may be NULL as well), and lf_attn_bwd, given
+ *   D = NULL, computes D itself for the rows of kept blocks.  With
+ *   LF_SELECT_NORMS_GIVEN and D = NULL no norm pass runs (dout may be NULL). */
 lf_status lf_block_select(const lf_attn_desc* desc, const void* dout, const void* o,
                           double delta, uint64_t seed, uint64_t step, uint32_t flags,
                           float* block_norm, float* D, double* tau, float* block_weight,
@@ -160,10 +163,17 @@ lf_status lf_block_select_rule(const lf_attn_desc* desc, const void* dout, const
  *   (summed over the hq/hkv query heads of a KV head), dV = P^T dO~.
  *   q, k, v, dout bf16 in (layouts as above); lse, D fp32 [hq][T] from
  *   lf_attn_fwd / lf_block_select (D may be NULL: it is then computed from o
- *   and dout into the workspace; o may be NULL when D is given);
+ *   and dout into the workspace, for the rows of kept blocks only, the others
+ *   being 0; o may be NULL when D is given);
  *   block_weight, kept_idx, kept_cnt from lf_block_select;
  *   dq [T][hq][d], dk, dv [T][hkv][d] bf16 out.  Rows of dropped blocks get
- *   dq = 0; dk/dv rows no kept block reaches get 0. */
+ *   dq = 0; dk/dv rows no kept block reaches get 0.  The rows of q and dout that
+ *   belong to dropped blocks are never read (at 64-row granularity when
+ *   block_q = 64), except rows that fall inside the last tile of the previous
+ *   segment (a segment's last 128-row tile, or 64-row half, also loads the rows
+ *   after the segment's end; they are masked with P = 0).  Inputs must be finite:
+ *   a non-finite value in those rows, or in the k/v rows after a segment's end
+ *   within its last tile, can turn the masked products into NaN. */
 lf_status lf_attn_bwd(const lf_attn_desc* desc, const void* q, const void* k, const void* v,
                       const void* o, const float* lse, const void* dout, const float* D,
                       const float* block_weight, const int32_t* kept_idx,
