@@ -242,6 +242,14 @@ lf_status launch_bwd(const lf_attn_desc* d, const void* q, const void* k, const 
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return LF_ERR_CUDA;
     dim3 grid(ntiles_of(d), d->hq / p.heads_per_cta, d->nseq);
+    // up to eight waves of CTAs per segment (16K tokens at 8 KV heads): every head
+    // group's heavy tiles first; longer segments run one group at a time, which keeps
+    // the group's Q, dO and dQ accumulator in L2 (the other order was slower at 32K)
+    int dev = 0, nsm = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return LF_ERR_CUDA;
+    p.tile_major = (long long)grid.x * grid.y <= 8LL * nsm ? 1 : 0;
     kern<<<grid, lf::kBwdThreads, smem, st>>>(mq, mk, mv, mdo, mdvacc, mdkacc, mq64, mdo64, p);
     if (launch_status() != LF_OK) return LF_ERR_CUDA;
     // fp32 accumulators -> bf16 results (dQ and dK take the softmax scale)

@@ -67,6 +67,9 @@ struct BwdParams {
     // when a CTA covers the whole query group of its KV head (kv_out_direct) they go
     // instead, final, to the bf16 outputs [T][hkv][D], zeroed by the caller
     int kv_out_direct;
+    // CTA order within a segment: 0 = KV tile fastest, one head group after another;
+    // 1 = head group fastest (every group's heavy low tiles start first)
+    int tile_major;
     __nv_bfloat16* dk_out;
     __nv_bfloat16* dv_out;
 };
@@ -232,10 +235,20 @@ __global__ void __launch_bounds__(kBwdThreads, 1)
     PairEntry* ring = reinterpret_cast<PairEntry*>(bars + 20);   // [4] x 16 B
     uint64_t* bar_acc0 = bars + 28;       // one phase: half 0's first dV/dK MMAs completed (!kHalves)
 
-    // KV tile fastest: CTAs resident together share one query head, so its Q,
-    // dO and dQ accumulator stay in L2; the lowest tiles (most work) start first
-    const int jt = blockIdx.x;
-    const int hgrp = blockIdx.y;            // query heads hgrp*G .. hgrp*G+G-1, G = heads_per_cta
+    // KV tile fastest: CTAs resident together share one head group, so its Q, dO and
+    // dQ accumulator stay in L2, and each group's lowest tiles (most work) start first.
+    // When a segment's CTAs make only a few waves, the last group's heaviest CTAs would
+    // start late and run alone at the end; there the group runs fastest instead, so
+    // that the heavy tiles of every group start first.
+    int jt, hgrp;                           // hgrp: query heads hgrp*G .. hgrp*G+G-1, G = heads_per_cta
+    if (prm.tile_major) {
+        const int lin = static_cast<int>(blockIdx.x + blockIdx.y * gridDim.x);
+        jt = lin / static_cast<int>(gridDim.y);
+        hgrp = lin % static_cast<int>(gridDim.y);
+    } else {
+        jt = blockIdx.x;
+        hgrp = blockIdx.y;
+    }
     const int s = blockIdx.z;
     int seg0, len;
     if (!load_segment(prm.cu_seqlens, s, prm.T, prm.max_seqlen, seg0, len, 30)) return;
