@@ -149,6 +149,13 @@ lf_status launch_fwd(const lf_attn_desc* d, const void* q, const void* k, const 
     // (x: pairs of query tiles over all segments, flattened; see segment_of_unit)
     const long long pair_units = ((long long)d->total_tokens + 255ll * d->nseq) >> 8;
     dim3 grid(static_cast<unsigned>(pair_units * (d->hq / d->hkv)), d->hkv, 1);
+    // up to eight waves: every KV head's longest rows first (the whole grid's K/V then
+    // shares L2, which is small at these lengths)
+    int dev = 0, nsm = 148;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return LF_ERR_CUDA;
+    p.tile_major = (long long)grid.x * grid.y <= 8LL * nsm ? 1 : 0;
     lf::attn_fwd_kernel<D><<<grid, lf::kFwdThreads, smem, st>>>(mq, mk, mv, p);
     return launch_status();
 }

@@ -34,6 +34,7 @@ struct FwdParams {
     const int32_t* cu_seqlens;
     int T, hq, hkv, causal, max_seqlen, nseq;
     float scale_log2;          // softmax_scale * log2(e)
+    int tile_major;            // CTA order: 1 = KV head fastest (see the kernel)
     __nv_bfloat16* o;
     float* lse;
 };
@@ -82,11 +83,21 @@ __global__ void __launch_bounds__(kFwdThreads, 1)
     // 256 query rows running over all segments, segment by segment; blockIdx.y = KV
     // head.  The G query heads that share a KV head run together, longest rows first
     // within each segment, so their K/V stay in L2 and each group's work outlasts its
-    // heaviest CTA.
+    // heaviest CTA.  With few waves of CTAs (tile_major) the KV head runs fastest
+    // instead, so that every KV head's longest rows start first rather than the last
+    // head's running alone at the end.
     const int G = prm.hq / prm.hkv;
-    const int g = blockIdx.y;
-    const int h = g * G + static_cast<int>(blockIdx.x) % G;
-    const int pg = static_cast<int>(blockIdx.x) / G;
+    int g, xr;
+    if (prm.tile_major) {
+        const int lin = static_cast<int>(blockIdx.x + blockIdx.y * gridDim.x);
+        g = lin % static_cast<int>(gridDim.y);
+        xr = lin / static_cast<int>(gridDim.y);
+    } else {
+        g = blockIdx.y;
+        xr = blockIdx.x;
+    }
+    const int h = g * G + xr % G;
+    const int pg = xr / G;
     const int s = segment_of_unit(prm.cu_seqlens, prm.nseq, pg, 8);
     if (s < 0) return;
     int seg0, len;
