@@ -667,13 +667,6 @@ def main():
     sets_buf = [bufs, lf.Buffers(desc, device=dev)]
     up, down = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
 
-    def step_on(din, b):
-        lf.lf_attn_fwd(desc, din["q"], din["k"], din["v"], b.o, b.lse)
-        lf.lf_block_select_rule(desc, din["dout"], b.o, rule_id, rule_param, 0, 0, 0, b.norm, b.D,
-                                b.tau, b.w, b.keep, b.kept_idx, b.kept_cnt)
-        lf.lf_attn_bwd(desc, din["q"], din["k"], din["v"], b.o, b.lse, din["dout"], b.D, b.w,
-                       b.kept_idx, b.kept_cnt, b.dq, b.dk, b.dv, b.ws)
-
     Ke = max(3, K)   # as many steps as the device-timed region
     if dist is not None:
         dist.barrier()
@@ -682,33 +675,51 @@ def main():
     e2e = torch.cuda.Event(enable_timing=True)
     e2s.record(stream)
     up.wait_event(e2s)
-    uploaded, computed, downloaded = [None, None], [None, None], [None, None]
+    # per set: q/k/v uploaded, dout uploaded, forward done, backward done, results out
+    up_qkv, up_do, fwd_done, computed, downloaded = ([None, None] for _ in range(5))
 
     def upload(i):
+        # the forward needs only q, k, v: dout follows, under the forward
         s_ = i % 2
         if computed[s_] is not None:          # step i-2 has finished reading this set
             up.wait_event(computed[s_])
         with torch.cuda.stream(up):
-            for k_, t in host.items():
-                sets_in[s_][k_].copy_(t, non_blocking=True)
-        uploaded[s_] = torch.cuda.Event()
-        uploaded[s_].record(up)
+            for k_ in ("q", "k", "v"):
+                sets_in[s_][k_].copy_(host[k_], non_blocking=True)
+            up_qkv[s_] = torch.cuda.Event()
+            up_qkv[s_].record(up)
+            sets_in[s_]["dout"].copy_(host["dout"], non_blocking=True)
+            up_do[s_] = torch.cuda.Event()
+            up_do[s_].record(up)
+
+    def download(s_, keys, after):
+        down.wait_event(after)
+        with torch.cuda.stream(down):
+            for k_ in keys:
+                h_out[s_][k_].copy_(getattr(sets_buf[s_], k_), non_blocking=True)
 
     upload(0)
     for i in range(Ke):
         s_ = i % 2
-        stream.wait_event(uploaded[s_])
+        din, b = sets_in[s_], sets_buf[s_]
         if downloaded[s_] is not None:        # step i-2's results have left this set
             stream.wait_event(downloaded[s_])
-        step_on(sets_in[s_], sets_buf[s_])
+        stream.wait_event(up_qkv[s_])
+        lf.lf_attn_fwd(desc, din["q"], din["k"], din["v"], b.o, b.lse)
+        fwd_done[s_] = torch.cuda.Event()
+        fwd_done[s_].record(stream)
+        stream.wait_event(up_do[s_])
+        lf.lf_block_select_rule(desc, din["dout"], b.o, rule_id, rule_param, 0, 0, 0, b.norm, b.D,
+                                b.tau, b.w, b.keep, b.kept_idx, b.kept_cnt)
+        lf.lf_attn_bwd(desc, din["q"], din["k"], din["v"], b.o, b.lse, din["dout"], b.D, b.w,
+                       b.kept_idx, b.kept_cnt, b.dq, b.dk, b.dv, b.ws)
         computed[s_] = torch.cuda.Event()
         computed[s_].record(stream)
         if i + 1 < Ke:
             upload(i + 1)
-        down.wait_event(computed[s_])
-        with torch.cuda.stream(down):
-            for k_, t in h_out[s_].items():
-                t.copy_(getattr(sets_buf[s_], k_), non_blocking=True)
+        # O and LSE leave under the selection and the backward; the gradients after it
+        download(s_, ("o", "lse"), fwd_done[s_])
+        download(s_, ("dq", "dk", "dv"), computed[s_])
         downloaded[s_] = torch.cuda.Event()
         downloaded[s_].record(down)
     stream.wait_event(downloaded[(Ke - 1) % 2])
@@ -786,7 +797,9 @@ def main():
                 "is": "backward executed FLOPs per second of data-fed step time (fwd, select, "
                       "bwd and the host copies of inputs and results)",
                 "copies": "pinned host buffers; uploads and downloads on two side streams, "
-                          "device inputs and outputs double-buffered"},
+                          "device inputs and outputs double-buffered; the forward starts once "
+                          "q, k, v are in (dout follows under it) and O, LSE leave under the "
+                          "backward"},
         "gpu_launches": kernels_per_step(w) * K,
         "clocks": clk,
     }
