@@ -164,11 +164,16 @@ __device__ __forceinline__ double warp_butterfly_sum(double v) {
 // ---------------------------------------------------------------------------
 constexpr int kSelectThreads = 256;
 
+// One block's term of the bisection's test at threshold t = mid, the test
+// multiplied through by t so that it takes no division.  RULE 0: the discarded
+// mass (1 - m/t) m becomes m t - m^2 (one fused multiply-add; the square of an
+// fp32 norm is exact in fp64), 0 for m >= t.  RULE 1: the keep probability
+// min(1, m/t) becomes min(t, m), exact.
 template <int RULE>
 __device__ __forceinline__ double select_term(float mf, double mid) {
     const double m = static_cast<double>(mf);
-    if (RULE == 0) return (m >= mid) ? 0.0 : __dmul_rn(__dsub_rn(1.0, __ddiv_rn(m, mid)), m);
-    return (m >= mid) ? 1.0 : __ddiv_rn(m, mid);
+    if (RULE == 0) return (m >= mid) ? 0.0 : __fma_rn(m, mid, -__dmul_rn(m, m));
+    return (m >= mid) ? mid : m;
 }
 
 // sum_i term(m_i, mid) in the pinned order (lane l: i = l, l + 32, ... in index
@@ -178,7 +183,7 @@ __device__ __forceinline__ double pinned_eval(const float* m_s, int n, double mi
     const int lane = threadIdx.x & 31;
     double acc = 0.0;
     int i = lane;
-    for (; i + 96 < n; i += 128) {   // four independent divides in flight, adds in order
+    for (; i + 96 < n; i += 128) {   // four independent terms in flight, adds in order
         const double t0 = select_term<RULE>(m_s[i], mid), t1 = select_term<RULE>(m_s[i + 32], mid);
         const double t2 = select_term<RULE>(m_s[i + 64], mid), t3 = select_term<RULE>(m_s[i + 96], mid);
         acc = __dadd_rn(acc, t0);
@@ -243,7 +248,8 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(
     const bool bisect = (RULE == 0 && param > 0.0 && total > 0.0) ||
                         (RULE == 1 && n > 0 && total > 0.0 && param < 1.0);
     if (bisect) {
-        // RULE 0: feasible iff f(mid) <= delta * M; RULE 1: iff g(mid) >= f * n
+        // RULE 0: feasible iff f(mid) <= delta * M; RULE 1: iff g(mid) >= f * n; both
+        // evaluated multiplied through by mid (sum of the terms above against crit * mid)
         const double crit = RULE == 0 ? __dmul_rn(param, total) : __dmul_rn(param, static_cast<double>(n));
         double lo = 0.0, hi = RULE == 0 ? __ddiv_rn(mx, __dsub_rn(1.0, param)) : __ddiv_rn(total, crit);
         for (int it = 0; it < 64;) {
@@ -258,8 +264,10 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(
                     const double mid = bisect_mid(l, u);
                     if ((node >> bit) & 1) l = mid; else u = mid;
                 }
-                const double v = pinned_eval<RULE>(m_s, n, bisect_mid(l, u));
-                if (lane == 0) flag_s[warp] = RULE == 0 ? (v <= crit) : (v >= crit);
+                const double t = bisect_mid(l, u);
+                const double v = pinned_eval<RULE>(m_s, n, t);
+                const double rhs = __dmul_rn(crit, t);
+                if (lane == 0) flag_s[warp] = RULE == 0 ? (v <= rhs) : (v >= rhs);
             }
             __syncthreads();
             int node = 1;

@@ -20,7 +20,8 @@
  *     (same section, second paragraph).
  * The precise reading used here: p_b = min(1, m_b / tau), tau the largest value
  * whose expected discarded mass sum_b (1 - p_b) m_b is at most delta * sum_b m_b,
- * found by 64 bisection steps; the draw is word 0 of Philox4x32-10 (Salmon,
+ * found by 64 bisection steps (each test multiplied through by the midpoint, so
+ * that it takes no division); the draw is word 0 of Philox4x32-10 (Salmon,
  * Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy as 1, 2, 3", SC'11)
  * keyed on the seed and countered on (block, head, segment, step); kept blocks
  * carry weight 1/p_b.
@@ -248,6 +249,22 @@ double lfo_discarded_mass(const double* m, int n, double tau, double* scratch)
     return lfo_pinned_sum(scratch, n);
 }
 
+/* The bisection's test at a threshold t > 0: is the expected discarded mass   */
+/* within the budget B?  The inequality sum_b [m_b < t] (1 - m_b/t) m_b <= B is */
+/* multiplied through by t, so that it takes no division:                       */
+/*   sum_b [m_b < t] (m_b t - m_b^2) <= B t.                                    */
+/* Each term is one fused multiply-add of m_b, t and -m_b^2 (the square is      */
+/* exact for fp32 norms), the sum takes the pinned order and B t is one rounded */
+/* product.  Any rounding would do for the definition; this one is fixed so     */
+/* that both implementations make identical bisection steps.                    */
+static int lfo_budget_met(const double* m, int n, double t, double B, double* scratch)
+{
+    for (int b = 0; b < n; ++b)
+        scratch[b] = (m[b] >= t) ? 0.0
+                   : (LFO_MUTANT == 6 ? m[b] * m[b] : fma(m[b], t, -(m[b] * m[b])));
+    return lfo_pinned_sum(scratch, n) <= B * t;
+}
+
 /* tau of one (segment, head): the largest feasible threshold, by bisection.   */
 /* Returns 0 when every block is kept outright (delta == 0 or no mass).         */
 double lfo_tau(const double* m, int n, double delta)
@@ -262,8 +279,7 @@ double lfo_tau(const double* m, int n, double delta)
         double lo = 0.0, hi = mx / (1.0 - delta);
         for (int it = 0; it < 64; ++it) {
             double mid = 0.5 * (lo + hi);
-            double f = lfo_discarded_mass(m, n, mid, scratch);
-            if (f <= B) lo = mid; else hi = mid;
+            if (lfo_budget_met(m, n, mid, B, scratch)) lo = mid; else hi = mid;
         }
         tau = lo;
     }
@@ -571,6 +587,15 @@ double lfo_expected_kept(const double* m, int n, double tau, double* scratch)
     return lfo_pinned_sum(scratch, n);
 }
 
+/* The fixed-fraction test at t > 0, multiplied through by t like the budget   */
+/* test: sum_b min(1, m_b/t) >= target becomes sum_b min(t, m_b) >= target t    */
+/* (every term exact; pinned order; target t one rounded product).              */
+static int lfo_count_met(const double* m, int n, double t, double target, double* scratch)
+{
+    for (int b = 0; b < n; ++b) scratch[b] = (m[b] >= t) ? t : m[b];
+    return lfo_pinned_sum(scratch, n) >= target * t;
+}
+
 double lfo_tau_fixed_fraction(const double* m, int n, double f)
 {
     double* scratch = (double*)malloc(sizeof(double) * (size_t)(n > 0 ? n : 1));
@@ -581,8 +606,7 @@ double lfo_tau_fixed_fraction(const double* m, int n, double f)
         double lo = 0.0, hi = M / target;
         for (int it = 0; it < 64; ++it) {
             double mid = 0.5 * (lo + hi);
-            double g = lfo_expected_kept(m, n, mid, scratch);
-            if (g >= target) lo = mid; else hi = mid;
+            if (lfo_count_met(m, n, mid, target, scratch)) lo = mid; else hi = mid;
         }
         tau = lo;
     }
