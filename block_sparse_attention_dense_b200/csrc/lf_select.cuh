@@ -155,10 +155,10 @@ __device__ __forceinline__ double warp_butterfly_sum(double v) {
 // min(1, m/tau)) from Philox and weight kept blocks 1/p.  RULE 2: top-k (k =
 // ceil(f * n)): the k largest norms (ties to the lower index), weight 1, no draw.
 //
-// The 64 bisection steps are taken three at a time: the seven midpoints the
-// next three steps can visit (a depth-3 tree below the current bracket, each
+// The 64 bisection steps are taken four at a time: the fifteen midpoints the
+// next four steps can visit (a depth-4 tree below the current bracket, each
 // computed by the same fp64 operations the sequential steps would use) are
-// evaluated at once, one warp each, every evaluation in the pinned summation
+// evaluated at once, two per warp, every evaluation in the pinned summation
 // order; the steps then follow the tree.  The result is the sequential
 // bisection's, bit for bit.
 // ---------------------------------------------------------------------------
@@ -195,6 +195,32 @@ __device__ __forceinline__ double pinned_eval(const float* m_s, int n, double mi
     return warp_butterfly_sum(acc);
 }
 
+// The same sums at two thresholds at once (two independent chains, each in the
+// pinned order).
+template <int RULE>
+__device__ __forceinline__ void pinned_eval2(const float* m_s, int n, double t0, double t1,
+                                             double& v0, double& v1) {
+    const int lane = threadIdx.x & 31;
+    double a0 = 0.0, a1 = 0.0;
+    int i = lane;
+    for (; i + 32 < n; i += 64) {
+        const float m0 = m_s[i], m1 = m_s[i + 32];
+        const double p0 = select_term<RULE>(m0, t0), q0 = select_term<RULE>(m0, t1);
+        const double p1 = select_term<RULE>(m1, t0), q1 = select_term<RULE>(m1, t1);
+        a0 = __dadd_rn(a0, p0);
+        a1 = __dadd_rn(a1, q0);
+        a0 = __dadd_rn(a0, p1);
+        a1 = __dadd_rn(a1, q1);
+    }
+    for (; i < n; i += 32) {
+        const float m0 = m_s[i];
+        a0 = __dadd_rn(a0, select_term<RULE>(m0, t0));
+        a1 = __dadd_rn(a1, select_term<RULE>(m0, t1));
+    }
+    v0 = warp_butterfly_sum(a0);
+    v1 = warp_butterfly_sum(a1);
+}
+
 __device__ __forceinline__ double bisect_mid(double lo, double hi) {
     return __dmul_rn(0.5, __dadd_rn(lo, hi));
 }
@@ -207,7 +233,7 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(
     int32_t* __restrict__ kept_idx, int32_t* __restrict__ kept_cnt) {
     extern __shared__ float m_s[];
     __shared__ double red_s[2];
-    __shared__ int flag_s[8];
+    __shared__ int flag_s[16];
     __shared__ int wcnt_s[2][kSelectThreads / 32];
     __shared__ uint32_t hist_s[256];
     __shared__ uint32_t radix_s[2];
@@ -252,22 +278,42 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(
         // evaluated multiplied through by mid (sum of the terms above against crit * mid)
         const double crit = RULE == 0 ? __dmul_rn(param, total) : __dmul_rn(param, static_cast<double>(n));
         double lo = 0.0, hi = RULE == 0 ? __ddiv_rn(mx, __dsub_rn(1.0, param)) : __ddiv_rn(total, crit);
+        // heap node j of the tree below (lo, hi): bit 1 of the path = the step moved lo
+        // up to its midpoint, bit 0 = hi down; the midpoint is formed by the same
+        // operations the sequential steps would take
+        auto node_mid = [&](int node) {
+            const int depth = 31 - __clz(node);
+            double l = lo, u = hi;
+            for (int bit = depth - 1; bit >= 0; --bit) {
+                const double mid = bisect_mid(l, u);
+                if ((node >> bit) & 1) l = mid; else u = mid;
+            }
+            return bisect_mid(l, u);
+        };
+        auto feasible = [&](double v, double t) {
+            const double rhs = __dmul_rn(crit, t);
+            return RULE == 0 ? (v <= rhs) : (v >= rhs);
+        };
         for (int it = 0; it < 64;) {
-            const int levels = min(3, 64 - it);
-            // heap node j = warp + 1 of the tree below (lo, hi): bit 1 of the path = the
-            // step moved lo up to its midpoint, bit 0 = hi down
-            if (warp < (1 << levels) - 1) {
-                const int node = warp + 1;
-                const int depth = 31 - __clz(node);
-                double l = lo, u = hi;
-                for (int bit = depth - 1; bit >= 0; --bit) {
-                    const double mid = bisect_mid(l, u);
-                    if ((node >> bit) & 1) l = mid; else u = mid;
+            // four steps per round: the fifteen nodes of a depth-4 tree, nodes warp + 1
+            // and warp + 9 per warp (64 = 16 rounds of 4)
+            const int levels = min(4, 64 - it);
+            const int nodes = (1 << levels) - 1;
+            const int n0 = warp + 1, n1 = warp + 9;
+            if (n0 <= nodes) {
+                const double t0 = node_mid(n0);
+                if (n1 <= nodes) {
+                    const double t1 = node_mid(n1);
+                    double v0, v1;
+                    pinned_eval2<RULE>(m_s, n, t0, t1, v0, v1);
+                    if (lane == 0) {
+                        flag_s[n0 - 1] = feasible(v0, t0);
+                        flag_s[n1 - 1] = feasible(v1, t1);
+                    }
+                } else {
+                    const double v0 = pinned_eval<RULE>(m_s, n, t0);
+                    if (lane == 0) flag_s[n0 - 1] = feasible(v0, t0);
                 }
-                const double t = bisect_mid(l, u);
-                const double v = pinned_eval<RULE>(m_s, n, t);
-                const double rhs = __dmul_rn(crit, t);
-                if (lane == 0) flag_s[warp] = RULE == 0 ? (v <= rhs) : (v >= rhs);
             }
             __syncthreads();
             int node = 1;
