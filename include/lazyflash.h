@@ -113,8 +113,11 @@ lf_status lf_attn_fwd(const lf_attn_desc* desc, const void* q, const void* k, co
  *   D[h][t] = sum_c dO[t][h][c] * O[t][h][c] (fp32, unweighted);
  *   tau[s][h] (fp64) = the largest threshold whose expected discarded mass
  *     sum_i (1 - min(1, m_i/tau)) m_i is <= delta * sum_i m_i, found by 64
- *     bisection steps on [0, max_i m_i / (1 - delta)] with a fixed fp64
- *     summation order; 0 when delta == 0 or all norms are 0 (keep all);
+ *     bisection steps on [0, max_i m_i / (1 - delta)]; each step tests the
+ *     inequality multiplied through by the midpoint t, sum_i [m_i < t]
+ *     (m_i t - m_i^2) <= (delta M) t, in fp64 with one fused multiply-add per
+ *     block and a fixed summation order, so that the result is reproducible
+ *     bit for bit; 0 when delta == 0 or all norms are 0 (keep all);
  *   p_i = min(1, m_i / tau) (1 when tau == 0); keep_i = 1 iff p_i >= 1 or
  *     u24 < p_i * 2^24, u24 = word 0 of Philox4x32-10(counter = (i, h, s,
  *     step mod 2^32), key = (seed lo 32, seed hi 32)) >> 8;
@@ -136,8 +139,9 @@ enum {
     LF_RULE_BUDGET = 0,          /* the LazyFlash rule of lf_block_select; param = delta in [0, 1) */
     LF_RULE_FIXED_FRACTION = 1,  /* param = f in (0, 1]: tau = the largest threshold whose expected
                                     kept count sum_i min(1, m_i/tau) reaches f * n (64 bisection
-                                    steps, same fixed summation order); same Philox draw and 1/p
-                                    weights as the budget rule; tau = 0 (keep all) when f = 1 */
+                                    steps, each testing sum_i min(t, m_i) >= (f n) t in the same
+                                    fixed order); same Philox draw and 1/p weights as the budget
+                                    rule; tau = 0 (keep all) when f = 1 */
     LF_RULE_TOPK = 2             /* param = f in (0, 1]: keep the k = ceil(f * n) largest norms
                                     (ties to the lower index) with weight 1, no draw; tau = the
                                     k-th largest norm */
