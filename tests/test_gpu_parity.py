@@ -41,6 +41,11 @@ SMALL = [
     # head-in-group index with an odd group
     synthetic.Workload("gqa3_d128", (333, 200), hq=6, hkv=2, d=128, block=128, sigma=1.5,
                        delta=0.1),
+    # exactly 32 query heads per KV head: the largest group one backward CTA walks
+    # whole (every head's start search and shared-memory slot in use, dK/dV stored
+    # directly as bf16), d = 128, two segments
+    synthetic.Workload("mqa_g32_d128", (300, 170), hq=32, hkv=1, d=128, block=128, sigma=1.5,
+                       delta=0.15),
     # 40 query heads per KV head: beyond the 32 heads one backward CTA walks, so two
     # CTAs share each KV tile and dK/dV meet in the fp32 accumulators
     synthetic.Workload("mqa_g40_d64", (300, 170), hq=40, hkv=1, d=64, block=128, sigma=1.5,
