@@ -91,6 +91,40 @@ def test_norms_and_rowdot_match_oracle(w):
     assert np.all(np.abs(D - D_ref) <= 1e-5 * scale + 1e-30)
 
 
+@pytest.mark.parametrize("w", [SMALL[2], SMALL[7]], ids=lambda w: w.name)
+def test_max_seqlen_above_the_longest_segment(w):
+    """max_seqlen is an upper bound on the segment lengths: three times the longest
+    (more KV-tile CTAs, forward work units and per-block slots than any segment uses)
+    gives the oracle's results, with the slots past each segment's blocks empty."""
+    inp = synthetic.make_inputs(w)
+    dev = to_dev(inp)
+    big = 3 * w.max_seqlen + 5
+    desc = lf.make_desc(dev["cu_seqlens"], big, w.total_tokens, w.hq, w.hkv, w.d, w.scale,
+                        w.causal, w.block)
+    bufs = lf.Buffers(desc)
+    lf.lazyflash_step(desc, dev["q"], dev["k"], dev["v"], dev["dout"], w.delta, 3, 1, bufs)
+    lf.lf_check_device_error()
+    torch.cuda.synchronize()
+    cu, nb = w.cu_seqlens(), nb_per_seq(w)
+    assert bufs.norm.shape[2] == (big + w.block - 1) // w.block
+    o_ref, lse_ref = oracle.attn_fwd(cu, inp["q"], inp["k"], inp["v"], w.scale, w.causal)
+    assert o_within(_cpu(bufs.o), o_ref, O_TOL)[0], o_within(_cpu(bufs.o), o_ref, O_TOL)
+    assert np.abs(_cpu(bufs.lse) - lse_ref).max() < LSE_TOL
+    m = _cpu(bufs.norm)
+    m_ref = oracle.block_norms(cu, inp["dout"], w.block, m.shape[2])
+    assert np.all(np.abs(m - m_ref) <= NORM_TOL * np.maximum(m_ref, 1e-30))
+    sel = oracle.select(m, nb, w.delta, 3, 1)
+    np.testing.assert_array_equal(bufs.keep.cpu().numpy(), sel["keep"])
+    np.testing.assert_array_equal(bufs.w.cpu().numpy(), sel["w"])
+    np.testing.assert_array_equal(bufs.kept_cnt.cpu().numpy(), sel["kept_cnt"])
+    dq_ref, dk_ref, dv_ref = oracle.attn_bwd(cu, inp["q"], inp["k"], inp["v"], inp["dout"],
+                                             w.scale, w.block, sel["w"].astype(np.float64),
+                                             w.causal)
+    assert rel_fro(_cpu(bufs.dq), dq_ref) < GRAD_TOL
+    assert rel_fro(_cpu(bufs.dk), dk_ref) < GRAD_TOL
+    assert rel_fro(_cpu(bufs.dv), dv_ref) < GRAD_TOL
+
+
 def _select_case(nseq_lens, hq, block, sigma, seed):
     w = synthetic.Workload("sel", tuple(nseq_lens), hq=hq, hkv=1 if hq % 2 else 2, d=64,
                            block=block, sigma=sigma, delta=0.1)
